@@ -1,0 +1,215 @@
+"""Seeded synthetic workloads for exact attention (prefill and KV-cache decode).
+
+This module only draws random tensors: it holds none of the attention arithmetic, so
+both the CPU oracle (through the tests) and the CUDA path consume exactly the same
+bf16 bits.  Shapes follow the notation of the pages' cost analysis (youngju.dev,
+"attention variants", section 1: B batch, H heads, N sequence length, d_k head dim)
+and their grouped-query layout (same page, section 2: q is (B, H, N, d_k), k/v are
+(B, G, N, d_k) with G key/value heads).  In this library G is called ``Hkv`` and the
+number of query heads per key/value head is ``R = Hq // Hkv``.
+
+Recipe (fixed so that every run and every machine sees the same bits):
+
+* one ``torch.Generator('cpu')`` per workload, seeded with ``seed``;
+* draw order: decode lengths -> per-head standard deviations -> Q -> K -> V ->
+  outlier key rows;
+* values are drawn as fp32 ``randn`` (times the per-head std or outlier factor, in
+  fp32) and cast once to bf16 (round to nearest even, as torch does).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+
+@dataclasses.dataclass
+class Prefill:
+    """One prefill problem: q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d), all bf16 on the CPU."""
+    name: str
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    causal: bool
+    scale: float
+    out_dtype: torch.dtype
+
+    @property
+    def shape(self):
+        B, Hq, Nq, d = self.q.shape
+        Hkv, Nk = self.k.shape[1], self.k.shape[2]
+        return B, Hq, Hkv, Nq, Nk, d
+
+    def pairs(self) -> int:
+        """Number of (query row, key) pairs that the mask allows, summed over B and Hq."""
+        B, Hq, Hkv, Nq, Nk, d = self.shape
+        return B * Hq * allowed_pairs(Nq, Nk, self.causal)
+
+    def flops(self) -> float:
+        """Algorithmic flops: 2*d for q.k plus 2*d for p*v, per allowed pair."""
+        return 4.0 * self.shape[5] * self.pairs()
+
+    def io_bytes(self) -> int:
+        """Bytes that must cross HBM at least once: read Q, K, V, write O and LSE."""
+        B, Hq, Hkv, Nq, Nk, d = self.shape
+        ob = 4 if self.out_dtype == torch.float32 else 2
+        return 2 * (B * Hq * Nq * d + 2 * B * Hkv * Nk * d) + ob * B * Hq * Nq * d + 4 * B * Hq * Nq
+
+
+@dataclasses.dataclass
+class Decode:
+    """One decode step: q (B,Hq,d), caches (B,Hkv,Nmax,d) bf16, seqlens int32[B]."""
+    name: str
+    q: torch.Tensor
+    kcache: torch.Tensor
+    vcache: torch.Tensor
+    seqlens: torch.Tensor
+    scale: float
+
+    @property
+    def shape(self):
+        B, Hq, d = self.q.shape
+        Hkv, Nmax = self.kcache.shape[1], self.kcache.shape[2]
+        return B, Hq, Hkv, Nmax, d
+
+    def cache_bytes(self) -> int:
+        """K and V bytes that the step must read: 2 tensors * Hkv * d * 2 B per cached token."""
+        B, Hq, Hkv, Nmax, d = self.shape
+        return int(self.seqlens.to(torch.int64).sum().item()) * Hkv * d * 2 * 2
+
+    def io_bytes(self) -> int:
+        """Cache bytes plus the q read and the bf16 o write."""
+        B, Hq, Hkv, Nmax, d = self.shape
+        return self.cache_bytes() + 2 * 2 * B * Hq * d + 4 * B
+
+    def flops(self) -> float:
+        B, Hq, Hkv, Nmax, d = self.shape
+        return 4.0 * Hq * d * float(self.seqlens.to(torch.int64).sum().item())
+
+
+def allowed_pairs(Nq: int, Nk: int, causal: bool) -> int:
+    """Pairs (i, j) with key j visible to query i.
+
+    Causal masks use bottom-right alignment (row i sees keys 0 .. i + Nk - Nq), which
+    requires Nq <= Nk; every row then sees i + Nk - Nq + 1 keys.
+    """
+    if not causal:
+        return Nq * Nk
+    assert Nq <= Nk
+    off = Nk - Nq
+    return Nq * (off + 1) + Nq * (Nq - 1) // 2
+
+
+def _randn(gen, shape, std=None):
+    x = torch.randn(shape, generator=gen, dtype=torch.float32)
+    if std is not None:
+        x.mul_(std)
+    return x
+
+
+def make_prefill(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, *, seed: int,
+                 causal: bool, scale: Optional[float] = None,
+                 out_dtype: torch.dtype = torch.bfloat16,
+                 head_std_range: Optional[tuple] = None,
+                 outlier_rows_frac: float = 0.0, outlier_factor: float = 3.0,
+                 name: str = "prefill") -> Prefill:
+    """Draw a seeded prefill problem.
+
+    head_std_range=(lo, hi): each Q head and each K and V head gets its own standard
+    deviation, uniform in [lo, hi], drawn before any tensor value.
+    outlier_rows_frac: per (b, kv head), round(frac * Nk) key rows chosen by a seeded
+    permutation are multiplied by ``outlier_factor`` in fp32 before the bf16 cast.
+    """
+    assert Hq % Hkv == 0
+    gen = torch.Generator("cpu")
+    gen.manual_seed(seed)
+    q_std = k_std = v_std = None
+    if head_std_range is not None:
+        lo, hi = head_std_range
+        q_std = (lo + (hi - lo) * torch.rand((Hq,), generator=gen)).view(1, Hq, 1, 1)
+        k_std = (lo + (hi - lo) * torch.rand((Hkv,), generator=gen)).view(1, Hkv, 1, 1)
+        v_std = (lo + (hi - lo) * torch.rand((Hkv,), generator=gen)).view(1, Hkv, 1, 1)
+    q = _randn(gen, (B, Hq, Nq, d), q_std)
+    k = _randn(gen, (B, Hkv, Nk, d), k_std)
+    v = _randn(gen, (B, Hkv, Nk, d), v_std)
+    if outlier_rows_frac > 0.0:
+        n_out = int(round(outlier_rows_frac * Nk))
+        for b in range(B):
+            for g in range(Hkv):
+                rows = torch.randperm(Nk, generator=gen)[:n_out]
+                k[b, g, rows, :] *= outlier_factor
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    return Prefill(name=name, q=q.to(torch.bfloat16), k=k.to(torch.bfloat16),
+                   v=v.to(torch.bfloat16), causal=causal, scale=float(scale),
+                   out_dtype=out_dtype)
+
+
+def make_decode(B: int, Hq: int, Hkv: int, Nmax: int, d: int, *, seed: int,
+                len_range: tuple, scale: Optional[float] = None,
+                name: str = "decode") -> Decode:
+    """Draw a seeded decode step; seqlens uniform on the inclusive range ``len_range``."""
+    assert Hq % Hkv == 0
+    gen = torch.Generator("cpu")
+    gen.manual_seed(seed)
+    lo, hi = len_range
+    seqlens = torch.randint(lo, hi + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+    q = _randn(gen, (B, Hq, d))
+    kc = _randn(gen, (B, Hkv, Nmax, d))
+    vc = _randn(gen, (B, Hkv, Nmax, d))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    return Decode(name=name, q=q.to(torch.bfloat16), kcache=kc.to(torch.bfloat16),
+                  vcache=vc.to(torch.bfloat16), seqlens=seqlens, scale=float(scale))
+
+
+# The five named workloads.  Sizes follow the pages' examples (H=32 and d_k=128 in the
+# cost analysis, G=8 in the grouped-query section, contexts from 2K up to 32K).
+WORKLOADS = {
+    1: "mha_fwd_b1_h2_n256_d64_noncausal_f32out",
+    2: "mha_causal_prefill_b8_h32_n2048_d128",
+    3: "gqa_causal_prefill_b4_hq32_hkv8_n8192_d128",
+    4: "gqa_causal_prefill_b1_hq32_hkv8_n32768_d128_headstd",
+    5: "gqa_decode_b32_hq32_hkv8_nmax8192_d128",
+}
+
+
+def workload(k: int):
+    """Return workload k (1..5) with seed 1000+k."""
+    seed = 1000 + k
+    name = WORKLOADS[k]
+    if k == 1:
+        return make_prefill(1, 2, 2, 256, 256, 64, seed=seed, causal=False,
+                            out_dtype=torch.float32, name=name)
+    if k == 2:
+        return make_prefill(8, 32, 32, 2048, 2048, 128, seed=seed, causal=True,
+                            outlier_rows_frac=0.01, outlier_factor=3.0, name=name)
+    if k == 3:
+        return make_prefill(4, 32, 8, 8192, 8192, 128, seed=seed, causal=True, name=name)
+    if k == 4:
+        return make_prefill(1, 32, 8, 32768, 32768, 128, seed=seed, causal=True,
+                            head_std_range=(0.5, 2.0), name=name)
+    if k == 5:
+        return make_decode(32, 32, 8, 8192, 128, seed=seed, len_range=(1024, 8192), name=name)
+    raise KeyError(k)
+
+
+def sample_rows(N: int, count: int, seed: int, tile: int = 128) -> torch.Tensor:
+    """Seeded sorted row sample that always holds 0, 1, N-1 and the tile edges (t*tile-1, t*tile)."""
+    fixed = {0, 1, N - 1}
+    for t in range(1, (N + tile - 1) // tile):
+        fixed.add(t * tile - 1)
+        fixed.add(t * tile)
+    fixed = {r for r in fixed if 0 <= r < N}
+    gen = torch.Generator("cpu")
+    gen.manual_seed(seed)
+    extra = max(0, count - len(fixed))
+    perm = torch.randperm(N, generator=gen)[: extra + len(fixed)].tolist()
+    rows = set(fixed)
+    for r in perm:
+        if len(rows) >= max(count, len(fixed)):
+            break
+        rows.add(r)
+    return torch.tensor(sorted(rows), dtype=torch.int32)

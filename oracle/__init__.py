@@ -1,0 +1,127 @@
+"""CPU oracle for exact attention -- TEST INFRASTRUCTURE, not part of the library.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+may import this package.  It shares no code with the CUDA path (``exact_io_aware_81_b200``)
+and never imports it; the two meet only through the seeded inputs.
+
+Contents:
+  * ``attn_fwd`` / ``decode`` / ``probs``: the fp64 two-pass definition, in plain C with
+    OpenMP (``attn_oracle.c``), called through ctypes.
+  * ``online.online_attention``: a restatement of the block-by-block online softmax
+    (youngju.dev "attention variants", section 3), used only to check that the online
+    and two-pass forms agree.
+  * ``split_kv.split_kv_decode``: split-KV partials combined by a log-sum-exp merge,
+    used only to check that any chunking gives the unsplit result.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile attn_oracle.c with gcc -O2 -fopenmp into oracle/_build/liboracle.so."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        D = ctypes.c_double
+        lib.oracle_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I, D, I, P, I, P, P]
+        lib.oracle_attn_fwd.restype = I
+        lib.oracle_attn_probs.argtypes = [P, P, I, I, I, I, I, I, D, I, P]
+        lib.oracle_attn_probs.restype = I
+        lib.oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, D, P, P]
+        lib.oracle_decode.restype = I
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = I
+        _lib = lib
+    return _lib
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    assert t.dtype == torch.bfloat16, t.dtype
+    return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.int16).numpy()).view(np.uint16)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float, causal: bool,
+             rows: Optional[torch.Tensor] = None):
+    """fp64 attention of bf16 q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d).
+
+    Returns (o, lse) as float64 torch tensors of shape (B,Hq,R,d) and (B,Hq,R), where R
+    is len(rows) if a row sample is given, else Nq.
+    """
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    if rows is not None:
+        rw = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+        nr = int(rw.shape[0])
+        rp = _ptr(rw)
+    else:
+        rw, nr, rp = None, Nq, None
+    o = np.empty((B, Hq, nr, d), dtype=np.float64)
+    lse = np.empty((B, Hq, nr), dtype=np.float64)
+    rc = _load().oracle_attn_fwd(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Nq, Nk, d,
+                                 float(scale), int(bool(causal)), rp, nr, _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attn_fwd rejected its arguments")
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def probs(q: torch.Tensor, k: torch.Tensor, scale: float, causal: bool) -> torch.Tensor:
+    """Softmax weights P (B,Hq,Nq,Nk) in fp64, for tiny problems."""
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    qb, kb = _bits(q), _bits(k)
+    p = np.empty((B, Hq, Nq, Nk), dtype=np.float64)
+    rc = _load().oracle_attn_probs(_ptr(qb), _ptr(kb), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                   int(bool(causal)), _ptr(p))
+    if rc != 0:
+        raise ValueError("oracle_attn_probs rejected its arguments")
+    return torch.from_numpy(p)
+
+
+def decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens: torch.Tensor,
+           scale: float):
+    """fp64 decode: q (B,Hq,d) against caches (B,Hkv,Nmax,d) up to seqlens[b]."""
+    B, Hq, d = q.shape
+    Hkv, Nmax = kcache.shape[1], kcache.shape[2]
+    qb, kb, vb = _bits(q), _bits(kcache), _bits(vcache)
+    sl = np.ascontiguousarray(seqlens.detach().cpu().numpy().astype(np.int32))
+    o = np.empty((B, Hq, d), dtype=np.float64)
+    lse = np.empty((B, Hq), dtype=np.float64)
+    rc = _load().oracle_decode(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(sl), B, Hq, Hkv, Nmax, d,
+                               float(scale), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_decode rejected its arguments")
+    return torch.from_numpy(o), torch.from_numpy(lse)

@@ -1,0 +1,225 @@
+/*
+ * attn_oracle.c -- CPU fp64 reference for exact scaled-dot-product attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library's product path links, loads or
+ * calls this file; only the test suite, the smoke check and the benchmark's CPU
+ * baseline do.  It shares no code, header, table or helper with the CUDA sources.
+ *
+ * What it computes is the plain definition of attention, two passes per query row,
+ * in double precision from the exactly converted bf16 inputs:
+ *
+ *   s_ij  = scale * sum_t q[i,t] * k[j,t]            over the keys j that row i may see
+ *   m_i   = max_j s_ij,   l_i = sum_j exp(s_ij - m_i)                     (pass 1)
+ *   o_i   = sum_j exp(s_ij - m_i) * v[j,:] / l_i                          (pass 2)
+ *   lse_i = m_i + ln l_i
+ *
+ * Sources: the definition softmax(Q K^T / sqrt(d_k)) V of youngju.dev "attention
+ * variants" section 1 (cost analysis) and its gqa_attention example in section 2; the
+ * masked softmax of the toolsku.com MHA module (masked_fill(mask==0, -inf) before
+ * softmax).  Grouped-query sharing follows the same section-2 example: K/V head g is
+ * repeated R = Hq/Hkv times with repeat_interleave, so query head h reads K/V head
+ * floor(h / R).  Readings where the pages are silent:
+ *   - causal with Nq != Nk is bottom-right aligned: row i sees keys j <= i + Nk - Nq;
+ *   - decode (one query row per sequence) sees every cached key j < L_b, unmasked;
+ *   - lse is the natural log of sum_j exp(s_ij), scale included;
+ *   - a row that sees no key (only L_b = 0 in decode) gives o = 0 and lse = -inf.
+ *
+ * Parallelism: OpenMP over independent (batch, head, row) triples; each row is
+ * computed start to finish by one thread, so the result does not depend on the
+ * thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* bf16 is the upper half of an IEEE binary32; the conversion to double is exact. */
+static double bf16_bits_to_double(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Number of keys that query row i may see (keys 0 .. count-1). */
+static long visible_keys(long i, long Nq, long Nk, int causal)
+{
+    if (!causal) return Nk;
+    long last = i + (Nk - Nq);          /* bottom-right aligned causal limit */
+    if (last >= Nk) last = Nk - 1;
+    return last < 0 ? 0 : last + 1;
+}
+
+/* One query row against keys [0, nkeys) of one K/V head; writes d outputs and lse. */
+static void attend_row(const uint16_t *qrow, const uint16_t *khead, const uint16_t *vhead,
+                       long nkeys, long d, double scale,
+                       double *qbuf, double *s, double *orow, double *lse)
+{
+    for (long t = 0; t < d; ++t) qbuf[t] = bf16_bits_to_double(qrow[t]);
+    for (long t = 0; t < d; ++t) orow[t] = 0.0;
+    if (nkeys <= 0) { *lse = -INFINITY; return; }
+
+    /* scores */
+    for (long j = 0; j < nkeys; ++j) {
+        const uint16_t *kr = khead + j * d;
+        double acc = 0.0;
+        for (long t = 0; t < d; ++t) acc += qbuf[t] * bf16_bits_to_double(kr[t]);
+        s[j] = scale * acc;
+    }
+    /* pass 1: row max and normaliser */
+    double m = s[0];
+    for (long j = 1; j < nkeys; ++j) if (s[j] > m) m = s[j];
+    double l = 0.0;
+    for (long j = 0; j < nkeys; ++j) l += exp(s[j] - m);
+    /* pass 2: normalised weights times V */
+    for (long j = 0; j < nkeys; ++j) {
+        double p = exp(s[j] - m) / l;
+        const uint16_t *vr = vhead + j * d;
+        for (long t = 0; t < d; ++t) orow[t] += p * bf16_bits_to_double(vr[t]);
+    }
+    *lse = m + log(l);
+}
+
+/*
+ * Prefill / generic forward.
+ *   q: (B,Hq,Nq,d) bf16 bits;  k, v: (B,Hkv,Nk,d) bf16 bits.
+ *   rows: optional list of nrows query-row indices applied to every (b, h); NULL means
+ *         all Nq rows (nrows is then ignored).
+ *   o: (B,Hq,R,d) doubles, lse: (B,Hq,R) doubles, R = nrows or Nq.
+ * Returns 0, or -1 on an argument error.
+ */
+int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                    int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                    double scale, int causal, const int32_t *rows, int nrows,
+                    double *o, double *lse)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    const long R = Hq / Hkv;
+    const long nr = rows ? nrows : Nq;
+    const long total = (long)B * Hq * nr;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *qbuf = (double *)malloc(sizeof(double) * (size_t)d);
+        double *s = (double *)malloc(sizeof(double) * (size_t)Nk);
+        if (!qbuf || !s) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long idx = 0; idx < total; ++idx) {
+                long r = idx % nr;
+                long bh = idx / nr;
+                long h = bh % Hq;
+                long b = bh / Hq;
+                long g = h / R;
+                long i = rows ? rows[r] : r;
+                if (i < 0 || i >= Nq) { continue; }
+                const uint16_t *qrow = q + (((long)b * Hq + h) * Nq + i) * d;
+                const uint16_t *kh = k + ((long)b * Hkv + g) * (long)Nk * d;
+                const uint16_t *vh = v + ((long)b * Hkv + g) * (long)Nk * d;
+                attend_row(qrow, kh, vh, visible_keys(i, Nq, Nk, causal), d, scale,
+                           qbuf, s, o + idx * d, lse + idx);
+            }
+        }
+        free(qbuf);
+        free(s);
+    }
+    return err ? -1 : 0;
+}
+
+/*
+ * Softmax weights P (B,Hq,Nq,Nk) for tiny problems, by the same two passes; masked
+ * entries are exactly 0.  Used only to check that each row of P sums to one.
+ */
+int oracle_attn_probs(const uint16_t *q, const uint16_t *k,
+                      int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                      double scale, int causal, double *p)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    const long R = Hq / Hkv;
+    for (long b = 0; b < B; ++b)
+        for (long h = 0; h < Hq; ++h)
+            for (long i = 0; i < Nq; ++i) {
+                long g = h / R;
+                const uint16_t *qrow = q + ((b * Hq + h) * Nq + i) * d;
+                const uint16_t *kh = k + (b * Hkv + g) * (long)Nk * d;
+                double *prow = p + ((b * Hq + h) * Nq + i) * (long)Nk;
+                long nk = visible_keys(i, Nq, Nk, causal);
+                for (long j = 0; j < Nk; ++j) prow[j] = 0.0;
+                if (nk <= 0) continue;
+                double m = -INFINITY;
+                for (long j = 0; j < nk; ++j) {
+                    double acc = 0.0;
+                    for (long t = 0; t < d; ++t)
+                        acc += bf16_bits_to_double(qrow[t]) * bf16_bits_to_double(kh[j * d + t]);
+                    prow[j] = scale * acc;
+                    if (prow[j] > m) m = prow[j];
+                }
+                double l = 0.0;
+                for (long j = 0; j < nk; ++j) l += exp(prow[j] - m);
+                for (long j = 0; j < nk; ++j) prow[j] = exp(prow[j] - m) / l;
+            }
+    return 0;
+}
+
+/*
+ * Decode over a KV cache: one query row per (b, h) against cached keys [0, L_b).
+ *   q: (B,Hq,d);  kcache, vcache: (B,Hkv,Nmax,d);  seqlens: int32[B] in [0, Nmax].
+ *   o: (B,Hq,d) doubles, lse: (B,Hq) doubles.
+ */
+int oracle_decode(const uint16_t *q, const uint16_t *kcache, const uint16_t *vcache,
+                  const int32_t *seqlens, int B, int Hq, int Hkv, int Nmax, int d,
+                  double scale, double *o, double *lse)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nmax <= 0 || d <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > Nmax) return -1;
+    const long R = Hq / Hkv;
+    const long total = (long)B * Hq;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *qbuf = (double *)malloc(sizeof(double) * (size_t)d);
+        double *s = (double *)malloc(sizeof(double) * (size_t)Nmax);
+        if (!qbuf || !s) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long idx = 0; idx < total; ++idx) {
+                long h = idx % Hq;
+                long b = idx / Hq;
+                long g = h / R;
+                const uint16_t *kh = kcache + ((long)b * Hkv + g) * (long)Nmax * d;
+                const uint16_t *vh = vcache + ((long)b * Hkv + g) * (long)Nmax * d;
+                attend_row(q + idx * d, kh, vh, seqlens[b], d, scale, qbuf, s,
+                           o + idx * d, lse + idx);
+            }
+        }
+        free(qbuf);
+        free(s);
+    }
+    return err ? -1 : 0;
+}
+
+/* Number of OpenMP threads a parallel region would use (for reporting). */
+int oracle_num_threads(void)
+{
+    int n = 1;
+#pragma omp parallel
+    {
+#pragma omp single
+        {
+#ifdef _OPENMP
+            extern int omp_get_num_threads(void);
+            n = omp_get_num_threads();
+#endif
+        }
+    }
+    return n;
+}

@@ -1,0 +1,309 @@
+"""Pins for the CPU oracle, checked against facts that do not come from the oracle itself.
+
+Each pin names what fixes it: a closed form of the softmax, a property stated on the
+pages, a library routine (torch's fp64 CPU scaled_dot_product_attention), hand-expanded
+arithmetic on tiny inputs, or a fixture under tests/golden/.  A mutation test at the end
+plants plausible mistakes in a copy of the oracle's C source and checks that the pins
+catch every one of them.
+"""
+import math
+import os
+import re
+import shutil
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from oracle.online import online_attention
+from oracle.split_kv import split_kv_decode
+from exact_io_aware_81_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16(x):
+    return x.to(torch.bfloat16)
+
+
+def _rand(shape, seed, std=1.0):
+    g = torch.Generator("cpu").manual_seed(seed)
+    return _bf16(torch.randn(shape, generator=g) * std)
+
+
+def _sdpa_ref(q, k, v, scale, causal):
+    """torch CPU fp64 SDPA with a bottom-right causal mask and GQA expansion."""
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    R = Hq // Hkv
+    qd = q.double()
+    kd = k.double().repeat_interleave(R, dim=1)
+    vd = v.double().repeat_interleave(R, dim=1)
+    mask = None
+    if causal:
+        i = torch.arange(Nq).view(-1, 1)
+        j = torch.arange(Nk).view(1, -1)
+        mask = j <= i + (Nk - Nq)
+    o = F.scaled_dot_product_attention(qd, kd, vd, attn_mask=mask, scale=scale)
+    s = torch.matmul(qd, kd.transpose(-1, -2)) * scale
+    if mask is not None:
+        s = s.masked_fill(~mask, float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    return o, lse
+
+
+# --------------------------------------------------------------------------- pins
+
+def pin_probs_rows_sum_to_one():
+    q = _rand((1, 2, 9, 16), 1)
+    k = _rand((1, 2, 13, 16), 2)
+    for causal in (False, True):
+        p = oracle.probs(q, k, 0.25, causal)
+        assert torch.allclose(p.sum(-1), torch.ones(1, 2, 9, dtype=torch.float64), atol=1e-12, rtol=0)
+        assert (p >= 0).all()
+        if causal:
+            i = torch.arange(9).view(-1, 1)
+            j = torch.arange(13).view(1, -1)
+            assert (p[..., ~(j <= i + 4)] == 0).all()
+
+
+def pin_constant_v():
+    q = _rand((2, 4, 37, 32), 3, 2.0)
+    k = _rand((2, 2, 41, 32), 4, 2.0)
+    c = _bf16(torch.linspace(-3, 3, 32))
+    v = c.view(1, 1, 1, 32).expand(2, 2, 41, 32).contiguous()
+    for causal in (False, True):
+        o, _ = oracle.attn_fwd(q, k, v, 0.2, causal)
+        assert torch.allclose(o, c.double().view(1, 1, 1, 32).expand_as(o), atol=1e-12, rtol=0)
+
+
+def pin_first_causal_row():
+    q = _rand((1, 3, 20, 16), 5)
+    k = _rand((1, 3, 20, 16), 6)
+    v = _rand((1, 3, 20, 16), 7)
+    o, lse = oracle.attn_fwd(q, k, v, 0.3, True)
+    assert torch.equal(o[:, :, 0, :], v[:, :, 0, :].double())
+    s00 = 0.3 * (q[:, :, 0, :].double() * k[:, :, 0, :].double()).sum(-1)
+    assert torch.allclose(lse[:, :, 0], s00, atol=1e-12, rtol=0)
+
+
+def pin_zero_keys_mean_of_visible_values():
+    Nq, Nk = 11, 17
+    q = _rand((1, 2, Nq, 8), 8)
+    k = torch.zeros((1, 2, Nk, 8), dtype=torch.bfloat16)
+    v = _rand((1, 2, Nk, 8), 9)
+    o, lse = oracle.attn_fwd(q, k, v, 0.5, True)
+    for i in range(Nq):
+        n = i + (Nk - Nq) + 1
+        assert torch.allclose(o[0, :, i], v[0, :, :n].double().mean(1), atol=1e-12, rtol=0)
+        assert abs(lse[0, 0, i].item() - math.log(n)) < 1e-12
+    o, lse = oracle.attn_fwd(q, k, v, 0.5, False)
+    assert torch.allclose(o[0], v[0].double().mean(1, keepdim=True).expand(2, Nq, 8), atol=1e-12, rtol=0)
+    assert torch.allclose(lse, torch.full_like(lse, math.log(Nk)), atol=1e-12, rtol=0)
+
+
+def pin_key_permutation_invariance():
+    q = _rand((1, 2, 7, 16), 10)
+    k = _rand((1, 2, 29, 16), 11)
+    v = _rand((1, 2, 29, 16), 12)
+    perm = torch.randperm(29, generator=torch.Generator().manual_seed(0))
+    o1, l1 = oracle.attn_fwd(q, k, v, 0.25, False)
+    o2, l2 = oracle.attn_fwd(q, k[:, :, perm], v[:, :, perm], 0.25, False)
+    assert torch.allclose(o1, o2, atol=1e-12, rtol=0)
+    assert torch.allclose(l1, l2, atol=1e-12, rtol=0)
+
+
+def pin_dominant_key():
+    d = 64
+    q = _rand((1, 1, 1, d), 13)
+    k = _rand((1, 1, 50, d), 14)
+    v = _rand((1, 1, 50, d), 15)
+    k[0, 0, 23] = q[0, 0, 0] * 8  # exact in bf16 (power-of-two scaling)
+    o, _ = oracle.attn_fwd(q, k, v, 1.0 / math.sqrt(d), False)
+    assert torch.allclose(o[0, 0, 0], v[0, 0, 23].double(), atol=1e-9, rtol=0)
+
+
+def pin_library_sdpa():
+    cases = [  # (B, Hq, Hkv, Nq, Nk, d, causal)
+        (2, 4, 4, 33, 33, 32, False),
+        (2, 4, 4, 33, 33, 32, True),
+        (1, 6, 2, 19, 45, 16, True),    # GQA, chunked-prefill shape (Nq < Nk)
+        (1, 8, 1, 24, 24, 64, True),    # MQA
+        (1, 3, 3, 1, 70, 128, False),
+    ]
+    for n, (B, Hq, Hkv, Nq, Nk, d, causal) in enumerate(cases):
+        q = _rand((B, Hq, Nq, d), 100 + n)
+        k = _rand((B, Hkv, Nk, d), 200 + n, 1.5)
+        v = _rand((B, Hkv, Nk, d), 300 + n)
+        scale = 1.0 / math.sqrt(d)
+        o, lse = oracle.attn_fwd(q, k, v, scale, causal)
+        ro, rl = _sdpa_ref(q, k, v, scale, causal)
+        assert torch.allclose(o, ro, atol=1e-12, rtol=0), (n, (o - ro).abs().max())
+        assert torch.allclose(lse, rl, atol=1e-12, rtol=0), n
+
+
+def pin_brute_force_tiny():
+    # Nq = 2, Nk = 3, d = 2, one head; every entry expanded by hand with math.exp.
+    qv = [[1.0, -0.5], [0.25, 2.0]]
+    kv = [[0.5, 1.0], [-1.0, 0.75], [2.0, -0.25]]
+    vv = [[1.0, 2.0], [-3.0, 0.5], [0.125, -1.0]]
+    scale = 0.7
+    q = torch.tensor(qv, dtype=torch.bfloat16).view(1, 1, 2, 2)
+    k = torch.tensor(kv, dtype=torch.bfloat16).view(1, 1, 3, 2)
+    v = torch.tensor(vv, dtype=torch.bfloat16).view(1, 1, 3, 2)
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, scale, causal)
+        for i in range(2):
+            nvis = 3 if not causal else i + 2  # bottom-right: row 0 sees keys 0,1; row 1 all
+            s = [scale * (qv[i][0] * kv[j][0] + qv[i][1] * kv[j][1]) for j in range(nvis)]
+            e = [math.exp(x) for x in s]
+            z = sum(e)
+            for t in range(2):
+                want = sum(e[j] * vv[j][t] for j in range(nvis)) / z
+                assert abs(o[0, 0, i, t].item() - want) < 1e-12
+            assert abs(lse[0, 0, i].item() - math.log(z)) < 1e-12
+
+
+def pin_gqa_equals_mha_after_repeat_interleave():
+    q = _rand((2, 8, 21, 32), 16)
+    k = _rand((2, 2, 30, 32), 17)
+    v = _rand((2, 2, 30, 32), 18)
+    for causal in (False, True):
+        o1, l1 = oracle.attn_fwd(q, k, v, 0.2, causal)
+        o2, l2 = oracle.attn_fwd(q, k.repeat_interleave(4, 1).contiguous(),
+                                 v.repeat_interleave(4, 1).contiguous(), 0.2, causal)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def pin_gqa_head_map_golden():
+    table = [tuple(map(int, ln.split())) for ln in open(os.path.join(GOLDEN, "gqa_head_map.txt"))
+             if ln.strip() and not ln.startswith("#")]
+    Hq, Hkv = 32, 8
+    q = _rand((1, Hq, 5, 16), 19)
+    k = _rand((1, Hkv, 9, 16), 20)
+    v = torch.zeros((1, Hkv, 9, 16), dtype=torch.bfloat16)
+    for g in range(Hkv):
+        v[0, g] = float(g + 1)
+    o, _ = oracle.attn_fwd(q, k, v, 0.25, True)
+    for h, g in table:
+        assert torch.allclose(o[0, h], torch.full((5, 16), float(g + 1), dtype=torch.float64),
+                              atol=1e-12, rtol=0), (h, g)
+
+
+def pin_causal_block_rule_golden():
+    rules = [ln.split() for ln in open(os.path.join(GOLDEN, "causal_block_rule.txt"))
+             if ln.strip() and not ln.startswith("#")]
+    T = 5  # block edge
+    N = 4 * T
+    q = _rand((1, 1, N, 8), 21)
+    k = _rand((1, 1, N, 8), 22)
+    p = oracle.probs(q, k, 0.5, True)[0, 0]
+    for i, j, rule in rules:
+        i, j = int(i), int(j)
+        blk = p[i * T:(i + 1) * T, j * T:(j + 1) * T] != 0
+        if rule == "skip":
+            assert not blk.any()
+        elif rule == "full":
+            assert blk.all()
+        else:
+            assert torch.equal(blk, torch.ones(T, T, dtype=torch.bool).tril())
+
+
+def pin_online_equals_two_pass():
+    q = _rand((1, 1, 45, 16), 23, 2.0)
+    k = _rand((1, 1, 70, 16), 24, 2.0)
+    v = _rand((1, 1, 70, 16), 25)
+    for causal in (False, True):
+        qq = q[0, 0, 25:] if causal else q[0, 0]      # causal needs Nq <= Nk
+        qt = qq.view(1, 1, *qq.shape)
+        o, lse = oracle.attn_fwd(qt, k, v, 0.3, causal)
+        for bq, bk, lazy in [(1, 1, None), (3, 3, None), (64, 64, None), (4, 7, 8 * math.log(2)),
+                             (16, 5, None)]:
+            oo, ll = online_attention(qq.double().numpy(), k[0, 0].double().numpy(),
+                                      v[0, 0].double().numpy(), 0.3, causal, bq, bk, lazy)
+            assert np.allclose(oo, o[0, 0].numpy(), atol=1e-12, rtol=0), (bq, bk, causal)
+            assert np.allclose(ll, lse[0, 0].numpy(), atol=1e-12, rtol=0)
+
+
+def pin_decode_matches_library_and_split_merge():
+    B, Hq, Hkv, Nmax, d = 3, 8, 2, 300, 32
+    w = inputs.make_decode(B, Hq, Hkv, Nmax, d, seed=7, len_range=(0, Nmax))
+    sl = torch.tensor([0, 1, 300], dtype=torch.int32)
+    o, lse = oracle.decode(w.q, w.kcache, w.vcache, sl, w.scale)
+    assert (o[0] == 0).all() and torch.isinf(lse[0]).all() and (lse[0] < 0).all()
+    for b in (1, 2):
+        L = int(sl[b])
+        ro, rl = _sdpa_ref(w.q[b:b + 1].unsqueeze(2), w.kcache[b:b + 1, :, :L].contiguous(),
+                           w.vcache[b:b + 1, :, :L].contiguous(), w.scale, False)
+        assert torch.allclose(o[b], ro[0, :, 0], atol=1e-12, rtol=0)
+        assert torch.allclose(lse[b], rl[0, :, 0], atol=1e-12, rtol=0)
+    for chunk in (1, 7, 64, 256, 300):
+        so, sll = split_kv_decode(w.q.double().numpy(), w.kcache.double().numpy(),
+                                  w.vcache.double().numpy(), sl.numpy(), w.scale, chunk)
+        assert np.allclose(so, o.numpy(), atol=1e-12, rtol=0), chunk
+        assert np.allclose(sll[1:], lse[1:].numpy(), atol=1e-12, rtol=0)
+        assert np.isneginf(sll[0]).all()
+
+
+def pin_row_sample_matches_full():
+    q = _rand((2, 4, 300, 64), 26)
+    k = _rand((2, 2, 300, 64), 27)
+    v = _rand((2, 2, 300, 64), 28)
+    rows = inputs.sample_rows(300, 20, seed=3)
+    o, l = oracle.attn_fwd(q, k, v, 0.125, True)
+    os_, ls = oracle.attn_fwd(q, k, v, 0.125, True, rows=rows)
+    assert torch.equal(o[:, :, rows.long()], os_) and torch.equal(l[:, :, rows.long()], ls)
+
+
+PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__[4:])
+def test_pin(pin):
+    pin()
+
+
+# ------------------------------------------------------------------- mutation test
+# Each mutant is one plausible slip in the oracle's C source.  The pins above must fail
+# on every one of them.
+MUTANTS = [
+    ("gqa index", "long g = h / R;\n                long i", "long g = h % Hkv;\n                long i"),
+    ("causal offset dropped", "long last = i + (Nk - Nq);", "long last = i;"),
+    ("causal off by one", "return last < 0 ? 0 : last + 1;", "return last < 0 ? 0 : last;"),
+    ("max sign", "l += exp(s[j] - m);\n", "l += exp(s[j] + m);\n"),
+    ("scale dropped", "s[j] = scale * acc;", "s[j] = acc;"),
+    ("lse without max", "*lse = m + log(l);", "*lse = log(l);"),
+    ("transposed k index", "const uint16_t *kr = khead + j * d;", "const uint16_t *kr = khead + j;"),
+    ("normaliser dropped", "double p = exp(s[j] - m) / l;", "double p = exp(s[j] - m);"),
+    ("last key dropped", "for (long j = 0; j < nkeys; ++j) {\n        double p", "for (long j = 0; j + 1 < nkeys; ++j) {\n        double p"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(name, old, new, monkeypatch):
+    src = open(oracle._SRC).read()
+    assert src.count(old) >= 1, name
+    mutated = src.replace(old, new)
+    with tempfile.TemporaryDirectory() as td:
+        c = os.path.join(td, "m.c")
+        so = os.path.join(td, "m.so")
+        open(c, "w").write(mutated)
+        subprocess.check_call(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", so, c, "-lm"])
+        import ctypes
+        lib = ctypes.CDLL(so)
+        P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        lib.oracle_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I, D, I, P, I, P, P]
+        lib.oracle_attn_probs.argtypes = [P, P, I, I, I, I, I, I, D, I, P]
+        lib.oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, D, P, P]
+        monkeypatch.setattr(oracle, "_lib", lib)
+        caught = []
+        for pin in PINS:
+            try:
+                pin()
+            except AssertionError:
+                caught.append(pin.__name__)
+        assert caught, f"no pin caught mutant '{name}'"
