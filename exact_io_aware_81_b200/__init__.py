@@ -5,7 +5,7 @@ in ``include/fa.h``).  This package holds the thin ctypes binding (``ops``), the
 step (``build``) and the seeded workload generators (``inputs``).  Nothing here computes
 attention on the CPU: when the CUDA library is missing, every call raises.
 """
-__all__ = ["fwd", "decode", "decode_workspace_size", "get_error", "FAError"]
+__all__ = ["fwd", "decode", "decode_workspace_size", "get_error", "set_wait_limit_ns", "FAError"]
 
 
 def __getattr__(name):

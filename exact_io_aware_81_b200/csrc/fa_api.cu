@@ -1,0 +1,359 @@
+// fa_api.cu -- the C ABI of libfa.so (declared in include/fa.h): argument validation,
+// TMA tensor-map encoding, kernel launches on the caller's stream, and the device error
+// word.  The library owns no device memory on the compute path; the caller passes every
+// buffer, including the decode workspace.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_common.cuh"
+#include "fa_decode_sm100.cuh"
+#include "fa_prefill_sm100.cuh"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+
+thread_local char g_msg[512] = "";
+unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+
+int fail(int status, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int ok()
+{
+    g_msg[0] = '\0';
+    return FA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------ device facts, cached
+
+struct DeviceInfo {
+    bool valid = false;
+    bool sm100 = false;
+    int num_sms = 0;
+    bool prefill_attr_set[2][2] = {{false, false}, {false, false}};
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device(int *dev, DeviceInfo **info)
+{
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (*dev < 0 || *dev >= kMaxDevices) return fail(FA_ERR_UNSUPPORTED, "device index %d", *dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &d = g_dev[*dev];
+    if (!d.valid) {
+        int major = 0, minor = 0, sms = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev);
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev);
+        if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+        d.sm100 = (major == 10 && minor == 0);
+        d.num_sms = sms;
+        d.valid = true;
+    }
+    *info = &d;
+    if (!d.sm100) return fail(FA_ERR_UNSUPPORTED, "libfa.so is built for sm_100a (B200) only");
+    return FA_OK;
+}
+
+// -------------------------------------------------------------- TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// A (D, rows, planes) bf16 tensor with 128-row boxes of 64 columns, 128-byte swizzle.
+int encode_rows_map(CUtensorMap *m, const void *base, int D, long long rows, long long planes)
+{
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return FA_OK;
+}
+
+// ------------------------------------------------------------------- prefill
+
+int validate_fwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                 int o_dtype)
+{
+    if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID, "null pointer argument");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0)
+        return fail(FA_ERR_INVALID, "sizes must be positive (B=%d Hq=%d Hkv=%d Nq=%d Nk=%d d=%d)",
+                    B, Hq, Hkv, Nq, Nk, d);
+    if (Hq % Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (causal && Nq > Nk) return fail(FA_ERR_INVALID, "causal attention needs Nq <= Nk (%d > %d)", Nq, Nk);
+    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(FA_ERR_INVALID, "scale must be finite and > 0");
+    if (o_dtype != FA_BF16 && o_dtype != FA_F32) return fail(FA_ERR_INVALID, "unknown output dtype %d", o_dtype);
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(FA_ERR_UNSUPPORTED, "q, k, v and o must be 16-byte aligned");
+    if ((long long)B * Hq > 0x7fffffffLL || (long long)B * Hkv * Nk > 0x7fffffffLL * 64LL)
+        return fail(FA_ERR_UNSUPPORTED, "problem too large");
+    return FA_OK;
+}
+
+template <int D, bool F32>
+int launch_prefill(const fa::PrefillParams &p, DeviceInfo *info, cudaStream_t st)
+{
+    using C = fa::prefill::Cfg<D>;
+    auto kern = fa::fa_prefill_kernel<D, F32>;
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        bool &set = info->prefill_attr_set[D == 128][F32];
+        if (!set) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 C::kSmemBytes);
+            if (e != cudaSuccess)
+                return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+            set = true;
+        }
+    }
+    const int grid = p.n_units < info->num_sms ? p.n_units : info->num_sms;
+    kern<<<grid, fa::prefill::kThreads, C::kSmemBytes, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
+    return FA_OK;
+}
+
+int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, float scale, int causal, int o_dtype, void *stream,
+             int selftest_timeout)
+{
+    int rc = validate_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, o_dtype);
+    if (rc != FA_OK) return rc;
+    int dev;
+    DeviceInfo *info;
+    if ((rc = current_device(&dev, &info)) != FA_OK) return rc;
+
+    fa::PrefillParams p;
+    memset(&p, 0, sizeof p);
+    if ((rc = encode_rows_map(&p.tm_q, q, d, Nq, (long long)B * Hq)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_k, k, d, Nk, (long long)B * Hkv)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, v, d, Nk, (long long)B * Hkv)) != FA_OK) return rc;
+    p.o = o;
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.R = Hq / Hkv;
+    p.causal = causal ? 1 : 0;
+    p.head_pair = (p.R % 2 == 0) ? 1 : 0;
+    const int tiles = (Nq + 127) / 128;
+    if (p.head_pair) {
+        p.T = tiles;
+        p.upt = B * Hkv * (p.R / 2);
+    } else {
+        p.T = (tiles + 1) / 2;
+        p.upt = B * Hq;
+    }
+    const long long units = (long long)p.T * p.upt;
+    if (units > 0x7fffffffLL) return fail(FA_ERR_UNSUPPORTED, "problem too large");
+    p.n_units = (int)units;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.wait_limit_ns = g_wait_limit_ns;
+    p.selftest_no_s_signal = selftest_timeout;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128) rc = o_dtype == FA_F32 ? launch_prefill<128, true>(p, info, st) : launch_prefill<128, false>(p, info, st);
+    else rc = o_dtype == FA_F32 ? launch_prefill<64, true>(p, info, st) : launch_prefill<64, false>(p, info, st);
+    if (rc != FA_OK) return rc;
+    return ok();
+}
+
+// -------------------------------------------------------------------- decode
+
+long long decode_splits(int Nmax) { return (Nmax + fa::decode::kChunk - 1) / fa::decode::kChunk; }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t decode_ws_bytes(int B, int Hq, int Nmax, int d)
+{
+    if (B <= 0 || Hq <= 0 || Nmax <= 0 || d <= 0) return 0;
+    const size_t S = (size_t)decode_splits(Nmax);
+    return align256((size_t)B * Hq * S * d * sizeof(float)) + align256((size_t)B * Hq * S * sizeof(float));
+}
+
+template <int D, int RG>
+void launch_split(const fa::DecodeParams &p, cudaStream_t st)
+{
+    dim3 grid(p.S_max, p.Hq / RG, p.B);
+    fa::fa_decode_split_kernel<D, RG><<<grid, fa::decode::kThreads, 0, st>>>(p);
+}
+
+template <int D>
+void launch_split_rg(const fa::DecodeParams &p, int rg, cudaStream_t st)
+{
+    switch (rg) {
+    case 8: launch_split<D, 8>(p, st); break;
+    case 4: launch_split<D, 4>(p, st); break;
+    case 2: launch_split<D, 2>(p, st); break;
+    default: launch_split<D, 1>(p, st); break;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int d, float scale, int causal, void *stream)
+{
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, FA_BF16, stream, 0);
+}
+
+int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+              int Hkv, int Nq, int Nk, int d, float scale, int causal, int o_dtype, void *stream)
+{
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, o_dtype, stream, 0);
+}
+
+int fa_fwd_selftest_timeout(const void *q, const void *k, const void *v, void *o, float *lse,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                            int causal, void *stream)
+{
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, FA_BF16, stream, 1);
+}
+
+size_t fa_decode_workspace_size(int B, int Hq, int Nmax, int d) { return decode_ws_bytes(B, Hq, Nmax, d); }
+
+int fa_decode(const void *q, const void *kcache, const void *vcache, const int *seqlens, void *o,
+              float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale, void *workspace,
+              size_t workspace_bytes, void *stream)
+{
+    if (!q || !kcache || !vcache || !seqlens || !o) return fail(FA_ERR_INVALID, "null pointer argument");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nmax <= 0 || d <= 0)
+        return fail(FA_ERR_INVALID, "sizes must be positive (B=%d Hq=%d Hkv=%d Nmax=%d d=%d)", B, Hq, Hkv, Nmax, d);
+    if (Hq % Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(FA_ERR_INVALID, "scale must be finite and > 0");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
+        return fail(FA_ERR_UNSUPPORTED, "q, kcache, vcache and o must be 16-byte aligned");
+    if (B > 65535 || decode_splits(Nmax) > 0x7fffffffLL)
+        return fail(FA_ERR_UNSUPPORTED, "B must be <= 65535");
+    const size_t need = decode_ws_bytes(B, Hq, Nmax, d);
+    if (!workspace || workspace_bytes < need)
+        return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned16(workspace)) return fail(FA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    int dev, rc;
+    DeviceInfo *info;
+    if ((rc = current_device(&dev, &info)) != FA_OK) return rc;
+
+    const int R = Hq / Hkv;
+    const int rg = (R % 8 == 0) ? 8 : (R % 4 == 0) ? 4 : (R % 2 == 0) ? 2 : 1;
+    if (Hq / rg > 65535) return fail(FA_ERR_UNSUPPORTED, "too many head groups");
+
+    fa::DecodeParams p;
+    memset(&p, 0, sizeof p);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.kc = static_cast<const __nv_bfloat16 *>(kcache);
+    p.vc = static_cast<const __nv_bfloat16 *>(vcache);
+    p.seqlens = seqlens;
+    p.S_max = (int)decode_splits(Nmax);
+    p.part_o = static_cast<float *>(workspace);
+    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                           align256((size_t)B * Hq * p.S_max * d * sizeof(float)));
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nmax = Nmax;
+    p.R = R;
+    p.scale_log2 = scale * 1.4426950408889634f;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128) launch_split_rg<128>(p, rg, st);
+    else launch_split_rg<64>(p, rg, st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
+    dim3 mgrid(Hq, B);
+    if (d == 128) fa::fa_decode_merge_kernel<128><<<mgrid, 128, 0, st>>>(p);
+    else fa::fa_decode_merge_kernel<64><<<mgrid, 128, 0, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int fa_get_error(void *stream)
+{
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+    unsigned int word = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&word, fa::g_error_word, sizeof word);
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
+    if (word) {
+        e = cudaMemcpyToSymbol(fa::g_error_word, &zero, sizeof zero);
+        if (e != cudaSuccess) return fail(FA_ERR_CUDA, "clearing the error word: %s", cudaGetErrorString(e));
+    }
+    if (word & fa::kErrTimeout) return fail(FA_ERR_TIMEOUT, "a kernel pipeline wait exceeded its time limit");
+    if (word & fa::kErrSeqlenRange) return fail(FA_ERR_DEVICE_ARG, "seqlens held a value outside [0, Nmax]");
+    return ok();
+}
+
+void fa_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns = ns ? ns : kDefaultWaitLimitNs; }
+
+const char *fa_status_str(int status)
+{
+    switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID: return "FA_ERR_INVALID";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_DEVICE_ARG: return "FA_ERR_DEVICE_ARG";
+    default: return "FA_ERR_UNKNOWN";
+    }
+}
+
+const char *fa_last_error_message(void) { return g_msg; }
+
+int fa_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// fa_common.cuh -- device error word and time-bounded waits shared by the kernels.
+#pragma once
+
+#include <cstdint>
+
+#include "ptx_sm100.cuh"
+
+namespace fa {
+
+// Bits of the device error word (read and cleared by fa_get_error).
+enum : unsigned int {
+    kErrTimeout = 1u,      // a pipeline wait exceeded its limit
+    kErrSeqlenRange = 2u,  // a decode length was outside [0, Nmax] and was clamped
+};
+
+// One word per process, in the library's own device memory.
+__device__ unsigned int g_error_word = 0;
+
+__device__ __forceinline__ void raise_error(unsigned int bit) { atomicOr(&g_error_word, bit); }
+
+// Per-CTA stop flag (in shared memory): set by the first role whose wait runs out, read
+// by every other role at each wait so that the whole CTA winds down together.
+struct StopFlag {
+    volatile int *flag;
+    uint64_t limit_ns;
+
+    __device__ __forceinline__ bool stopped() const { return *flag != 0; }
+    __device__ __forceinline__ void stop() const { *flag = 1; }
+};
+
+// Wait by one thread for the phase of `bar` with parity `parity`.  Returns false if the
+// CTA was told to stop or the limit ran out (which records kErrTimeout and tells the
+// CTA to stop).
+__device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t parity, const StopFlag &sf)
+{
+    if (ptx::mbar_test(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (ptx::mbar_test(bar, parity)) return true;
+        if ((n & 31u) == 0u) {
+            if (sf.stopped()) return false;
+            if (ptx::globaltimer_ns() - t0 > sf.limit_ns) {
+                raise_error(kErrTimeout);
+                sf.stop();
+                return false;
+            }
+        }
+    }
+}
+
+// The same wait made by all 32 lanes of a warp together; the outcome is warp-uniform,
+// so that warp-collective tensor-memory instructions after it stay converged.
+__device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const StopFlag &sf)
+{
+    if (__all_sync(0xffffffffu, ptx::mbar_test(bar, parity))) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (__all_sync(0xffffffffu, ptx::mbar_test(bar, parity))) return true;
+        if ((n & 31u) == 0u) {
+            int give_up = 0;
+            if ((threadIdx.x & 31u) == 0u) {
+                if (sf.stopped()) {
+                    give_up = 1;
+                } else if (ptx::globaltimer_ns() - t0 > sf.limit_ns) {
+                    raise_error(kErrTimeout);
+                    sf.stop();
+                    give_up = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+        }
+    }
+}
+
+}  // namespace fa

@@ -1,0 +1,473 @@
+// fa_prefill_sm100.cuh -- exact attention forward (prefill) for sm_100a.
+//
+// Method (youngju.dev "attention variants", section 3 FlashAttention; toolsku.com,
+// generation 4): Q, K and V are cut into 128-row tiles that are staged into shared memory;
+// for each query tile the key/value tiles are visited in order, a block of scores is
+// formed on chip, and the softmax is accumulated online (running row maximum, running
+// sum, rescale of the partial output when the maximum moves).  Only O and the row
+// log-sum-exp go back to HBM; the (N, N) score matrix never exists in memory.  Causal
+// masks skip key tiles wholly in the future, mask the tiles that cross the diagonal and
+// compute the others in full (youngju.dev section 5.5).  Grouped-query heads share each
+// staged key/value tile (youngju.dev section 2; toolsku.com generation 2).
+//
+// B200 mapping (one persistent CTA per SM, 12 warps = 3 warpgroups):
+//   warp 8      TMA producer: Q tiles once per work unit, K_j / V_j into an NSTAGE ring
+//               of 128-byte-swizzled tiles, completion counted on mbarriers.
+//   warp 9      MMA issuer: S_s = Q_s K_j^T (both operands from shared memory) and
+//               O_s += P_s V_j (P from tensor memory, V from shared memory) with
+//               tcgen05.mma; accumulators live in tensor memory (512 columns:
+//               S0 | S1 | O0 | O1, P_s packed as bf16 over the first 64 columns of S_s).
+//   warps 0-3   softmax for Q tile 0, warps 4-7 for Q tile 1 (one thread per row):
+//               load S_s from TMEM, mask, row max, exp2 with the scale folded in
+//               (p = 2^(s*scale*log2e - m)), lazy rescale (the reference maximum is only
+//               moved when the new one exceeds it by more than 8 in log2 units; O_s is
+//               then rescaled in TMEM by the same warp), P_s to TMEM as bf16, fp32 row
+//               sum; at the end of a unit O_s / l and LSE are written out.
+//   warps 10-11 idle (they complete the third warpgroup).
+// The two Q tiles of a work unit share their key/value head: two query heads of one
+// group (R even) or two consecutive row tiles of one head (otherwise).  Their MMAs are
+// interleaved S0_j, PV1_{j-1}, S1_j, PV0_j so that the tensor core works on one tile
+// while the softmax warps work on the other.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "fa_common.cuh"
+#include "ptx_sm100.cuh"
+
+namespace fa {
+
+struct PrefillParams {
+    CUtensorMap tm_q;  // (d, Nq, B*Hq) bf16, box (64, 128, 1), 128B swizzle
+    CUtensorMap tm_k;  // (d, Nk, B*Hkv)
+    CUtensorMap tm_v;  // (d, Nk, B*Hkv)
+    void *o;
+    float *lse;
+    int B, Hq, Hkv, Nq, Nk;
+    int R;           // Hq / Hkv
+    int causal;
+    int head_pair;   // 1: a unit = heads (2p, 2p+1) of one group on the same 128 rows
+    int n_units;
+    int T;           // tile rows: 128-row tiles (head_pair) or 256-row tile pairs
+    int upt;         // units per tile row
+    float scale_log2;  // scale * log2(e)
+    unsigned long long wait_limit_ns;
+    int selftest_no_s_signal;  // timeout self-test: never signal a ready score tile
+};
+
+namespace prefill {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int kThreads = 384;   // 3 warpgroups
+constexpr int kChunkBytes = 128 * 128;  // one 64-column (128-byte) slab of a 128-row tile
+constexpr float kLazyThreshold = 8.0f;  // log2 units: rescale only past a factor of 256
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D>
+struct Cfg {
+    static constexpr int kTileBytes = 128 * D * 2;
+    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kQOff = 0;
+    static constexpr int kKVOff = 2 * kTileBytes;
+    static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+    // barriers: kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], p_ready[2],
+    //           o_done[2], o_free[2], teardown
+    static constexpr int kNumBars = 2 * kStages + 13;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
+};
+
+struct Unit {
+    int b, g, h0, h1, r0, r1, n0, n1;
+};
+
+__device__ __forceinline__ Unit decode_unit(const PrefillParams &p, int u)
+{
+    Unit w;
+    const int tr = u / p.upt;
+    const int rem = u - tr * p.upt;
+    const int t = p.causal ? (p.T - 1 - tr) : tr;  // causal: heaviest tile rows first
+    if (p.head_pair) {
+        const int hpairs = p.R >> 1;
+        const int hp = rem % hpairs;
+        const int bg = rem / hpairs;
+        w.g = bg % p.Hkv;
+        w.b = bg / p.Hkv;
+        w.h0 = w.g * p.R + 2 * hp;
+        w.h1 = w.h0 + 1;
+        w.r0 = w.r1 = BM * t;
+    } else {
+        const int h = rem % p.Hq;
+        w.b = rem / p.Hq;
+        w.g = h / p.R;
+        w.h0 = w.h1 = h;
+        w.r0 = 2 * BM * t;
+        w.r1 = w.r0 + BM;
+    }
+    const int nkt = (p.Nk + BN - 1) / BN;
+    if (p.causal) {
+        const int delta = p.Nk - p.Nq;
+        // the last row of a tile, r + 127, sees keys up to r + 127 + delta
+        w.n0 = min(nkt, (w.r0 + BM - 1 + delta) / BN + 1);
+        w.n1 = min(nkt, (w.r1 + BM - 1 + delta) / BN + 1);
+    } else {
+        w.n0 = w.n1 = nkt;
+    }
+    return w;
+}
+
+// S = Q K^T over the full head dimension: D/16 MMAs of K = 16.  Both operands are
+// K-major 128-byte-swizzled tiles: 8-row groups 1024 bytes apart (stride offset), a
+// K step of 16 elements advances the start address by 32 bytes inside the swizzle
+// atom, and the second 64-column slab (D = 128) starts 16 KB further on.
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_saddr, uint32_t k_saddr)
+{
+    constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, BN, 0);
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * kChunkBytes + (k & 3) * 32;
+        const uint64_t a = ptx::smem_desc_sw128(q_saddr + off, 16, 1024);
+        const uint64_t b = ptx::smem_desc_sw128(k_saddr + off, 16, 1024);
+        ptx::mma_ss(d_tmem, a, b, idesc, k > 0 ? 1u : 0u);
+    }
+}
+
+// O (+)= P V: 8 MMAs of K = 16 keys.  P (128 x 128 bf16) is read from tensor memory, 8
+// columns per K step.  V is an MN-major (d contiguous) 128-byte-swizzled tile: 8-key
+// groups 1024 bytes apart (stride offset), 64-column slabs of d 16 KB apart (leading
+// offset), and a K step of 16 keys advances 2048 bytes.
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_saddr,
+                                         bool accumulate)
+{
+    constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, D, 1);
+#pragma unroll
+    for (int k = 0; k < BN / 16; ++k) {
+        const uint64_t b = ptx::smem_desc_sw128(v_saddr + k * 2048, kChunkBytes, 1024);
+        ptx::mma_ts(d_tmem, p_tmem + k * 8, b, idesc, (accumulate || k > 0) ? 1u : 0u);
+    }
+}
+
+// A wait that ignores the stop flag, used only to let copies and MMAs already in
+// flight finish before the CTA leaves.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
+{
+    if (ptx::mbar_test(bar, parity)) return;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (!ptx::mbar_test(bar, parity)) {
+        if (ptx::globaltimer_ns() - t0 > limit_ns) {
+            raise_error(kErrTimeout);
+            return;
+        }
+    }
+}
+
+}  // namespace prefill
+
+template <int D, bool OUT_F32>
+__global__ void __launch_bounds__(prefill::kThreads, 1)
+    fa_prefill_kernel(const __grid_constant__ PrefillParams p)
+{
+    using namespace prefill;
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *kv_full = bars;
+    uint64_t *kv_empty = bars + C::kStages;
+    uint64_t *q_full = bars + 2 * C::kStages;
+    uint64_t *q_empty = q_full + 2;
+    uint64_t *s_full = q_full + 4;
+    uint64_t *p_ready = q_full + 6;
+    uint64_t *o_done = q_full + 8;
+    uint64_t *o_free = q_full + 10;
+    uint64_t *teardown = q_full + 12;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
+    int *stop_flag = reinterpret_cast<int *>(smem + C::kMiscOff + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::kStages; ++i) {
+            ptx::mbar_init(&kv_full[i], 1);
+            ptx::mbar_init(&kv_empty[i], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(&q_full[s], 1);
+            ptx::mbar_init(&q_empty[s], 1);
+            ptx::mbar_init(&s_full[s], 1);
+            ptx::mbar_init(&p_ready[s], 128);
+            ptx::mbar_init(&o_done[s], 1);
+            ptx::mbar_init(&o_free[s], 128);
+        }
+        ptx::mbar_init(teardown, 1);
+        *stop_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    if (warp == 9) {
+        ptx::tmem_alloc(tmem_holder, 512);
+        ptx::tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        ptx::tma_prefetch_desc(&p.tm_q);
+        ptx::tma_prefetch_desc(&p.tm_k);
+        ptx::tma_prefetch_desc(&p.tm_v);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const StopFlag sf{stop_flag, p.wait_limit_ns};
+
+    const uint32_t q_saddr0 = ptx::smem_addr(smem + C::kQOff);
+    const uint32_t kv_saddr0 = ptx::smem_addr(smem + C::kKVOff);
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t kv_it = 0, q_it = 0;
+            uint32_t q_fills[2] = {0u, 0u};
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+                const Unit w = decode_unit(p, u);
+                for (int s = 0; s < 2 && ok; ++s) {
+                    if (!wait_one(&q_empty[s], (q_it & 1u) ^ 1u, sf)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
+                    ++q_fills[s];
+                    const int h = s ? w.h1 : w.h0;
+                    const int r = s ? w.r1 : w.r0;
+                    uint8_t *dst = smem + C::kQOff + s * C::kTileBytes;
+#pragma unroll
+                    for (int c = 0; c < D / 64; ++c)
+                        ptx::tma_load_3d(dst + c * kChunkBytes, &p.tm_q, &q_full[s], 64 * c, r,
+                                         w.b * p.Hq + h);
+                }
+                if (!ok) break;
+                ++q_it;
+                const int plane = w.b * p.Hkv + w.g;
+                for (int j = 0; j < w.n1 && ok; ++j) {
+                    for (int kv = 0; kv < 2; ++kv) {
+                        const uint32_t st = kv_it % C::kStages;
+                        const uint32_t ph = (kv_it / C::kStages) & 1u;
+                        if (!wait_one(&kv_empty[st], ph ^ 1u, sf)) { ok = false; break; }
+                        ptx::mbar_arrive_expect_tx(&kv_full[st], C::kTileBytes);
+                        uint8_t *dst = smem + C::kKVOff + st * C::kTileBytes;
+                        const CUtensorMap *map = kv ? &p.tm_v : &p.tm_k;
+#pragma unroll
+                        for (int c = 0; c < D / 64; ++c)
+                            ptx::tma_load_3d(dst + c * kChunkBytes, map, &kv_full[st], 64 * c,
+                                             BN * j, plane);
+                        ++kv_it;
+                    }
+                }
+            }
+            // Let every copy this thread started land before the CTA can exit.
+            for (uint32_t st = 0; st < (uint32_t)C::kStages && st < kv_it; ++st) {
+                const uint32_t last = kv_it - 1 - ((kv_it - 1 - st) % C::kStages);
+                drain_wait(&kv_full[st], (last / C::kStages) & 1u, p.wait_limit_ns);
+            }
+            for (int s = 0; s < 2; ++s)
+                if (q_fills[s] > 0) drain_wait(&q_full[s], (q_fills[s] - 1) & 1u, p.wait_limit_ns);
+        }
+    } else if (warp == 9) {
+        // --------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            uint32_t kv_it = 0, units = 0;
+            uint32_t p_ph[2] = {0u, 0u};
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+                const Unit w = decode_unit(p, u);
+                const uint32_t q_par = units & 1u;
+                const uint32_t free_par = q_par ^ 1u;  // first unit passes at once
+                if (!wait_one(&q_full[0], q_par, sf) || !wait_one(&q_full[1], q_par, sf)) break;
+                ptx::tc_fence_after();
+                uint32_t prev_v = 0;
+                for (int j = 0; j < w.n1; ++j) {
+                    const uint32_t ks = kv_it % C::kStages;
+                    const uint32_t kph = (kv_it / C::kStages) & 1u;
+                    const uint32_t vs = (kv_it + 1) % C::kStages;
+                    const uint32_t vph = ((kv_it + 1) / C::kStages) & 1u;
+                    if (!wait_one(&kv_full[ks], kph, sf)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t k_saddr = kv_saddr0 + ks * C::kTileBytes;
+                    if (j < w.n0) {
+                        issue_qk<D>(tmem + 0, q_saddr0, k_saddr);
+                        if (!p.selftest_no_s_signal) ptx::mma_commit(&s_full[0]);
+                        if (j == w.n0 - 1) ptx::mma_commit(&q_empty[0]);
+                    }
+                    if (j > 0) {
+                        if (!wait_one(&p_ready[1], p_ph[1], sf)) { ok = false; break; }
+                        p_ph[1] ^= 1u;
+                        if (j - 1 == 0 && !wait_one(&o_free[1], free_par, sf)) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        issue_pv<D>(tmem + 384, tmem + 128, kv_saddr0 + prev_v * C::kTileBytes, j - 1 > 0);
+                        ptx::mma_commit(&kv_empty[prev_v]);
+                    }
+                    issue_qk<D>(tmem + 128, q_saddr0 + C::kTileBytes, k_saddr);
+                    if (!p.selftest_no_s_signal) ptx::mma_commit(&s_full[1]);
+                    ptx::mma_commit(&kv_empty[ks]);
+                    if (j == w.n1 - 1) ptx::mma_commit(&q_empty[1]);
+                    if (!wait_one(&kv_full[vs], vph, sf)) { ok = false; break; }
+                    if (j < w.n0) {
+                        if (!wait_one(&p_ready[0], p_ph[0], sf)) { ok = false; break; }
+                        p_ph[0] ^= 1u;
+                        if (j == 0 && !wait_one(&o_free[0], free_par, sf)) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        issue_pv<D>(tmem + 256, tmem + 0, kv_saddr0 + vs * C::kTileBytes, j > 0);
+                        if (j == w.n0 - 1) ptx::mma_commit(&o_done[0]);
+                    }
+                    prev_v = vs;
+                    kv_it += 2;
+                }
+                if (!ok) break;
+                // last P V of tile 1
+                if (!wait_one(&p_ready[1], p_ph[1], sf)) break;
+                p_ph[1] ^= 1u;
+                if (w.n1 == 1 && !wait_one(&o_free[1], free_par, sf)) break;
+                ptx::tc_fence_after();
+                issue_pv<D>(tmem + 384, tmem + 128, kv_saddr0 + prev_v * C::kTileBytes, w.n1 > 1);
+                ptx::mma_commit(&kv_empty[prev_v]);
+                ptx::mma_commit(&o_done[1]);
+                ++units;
+            }
+            // Every MMA and commit issued above completes before the CTA can exit.
+            ptx::mma_commit(teardown);
+            drain_wait(teardown, 0, p.wait_limit_ns);
+        }
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ softmax warps
+        const int s = warp >> 2;              // which Q tile of the unit
+        const int tid = threadIdx.x & 127;    // row inside the tile = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + 128u * s;        // S_s, and P_s over it
+        const uint32_t tO = tmem + lane_base + 256u + 128u * s;  // O_s
+        const float sl2 = p.scale_log2;
+        uint32_t s_ph = 0, units = 0;
+        for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+            const Unit w = decode_unit(p, u);
+            const int h = s ? w.h1 : w.h0;
+            const int r0 = s ? w.r1 : w.r0;
+            const int n = s ? w.n1 : w.n0;
+            const int row = r0 + tid;
+            const int lim = p.causal ? min(row + (p.Nk - p.Nq), p.Nk - 1) : p.Nk - 1;
+            float m = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < n; ++j) {
+                if (!wait_warp(&s_full[s], s_ph, sf)) { ok = false; break; }
+                s_ph ^= 1u;
+                ptx::tc_fence_after();
+                uint32_t x[128];
+                ptx::tmem_ld32(tS + 0, &x[0]);
+                ptx::tmem_ld32(tS + 32, &x[32]);
+                ptx::tmem_ld32(tS + 64, &x[64]);
+                ptx::tmem_ld32(tS + 96, &x[96]);
+                ptx::tmem_wait_ld();
+                const int kbase = BN * j;
+                if (kbase + BN - 1 > lim) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (kbase + c > lim) x[c] = __float_as_uint(-INFINITY);
+                }
+                float mx = __uint_as_float(x[0]);
+#pragma unroll
+                for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(x[c]));
+                const float m_new = fmaxf(m, mx * sl2);
+                float alpha = 1.f;
+                bool rescale = false;
+                if (j == 0) {
+                    m = m_new;
+                } else if (m_new - m > kLazyThreshold) {
+                    alpha = ptx::ex2(m - m_new);
+                    m = m_new;
+                    rescale = true;
+                }
+                // P = 2^(s * scale * log2e - m), packed in place as bf16 pairs.
+                const float negm = -m;
+                float sum = 0.f;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const float p0 = ptx::ex2(fmaf(__uint_as_float(x[2 * c]), sl2, negm));
+                    const float p1 = ptx::ex2(fmaf(__uint_as_float(x[2 * c + 1]), sl2, negm));
+                    sum += p0 + p1;
+                    x[c] = ptx::pack_bf16x2(p0, p1);
+                }
+                ptx::tmem_st32(tS + 0, &x[0]);
+                ptx::tmem_st32(tS + 32, &x[32]);
+                // Rare (lazy) rescale of the partial output, before P V of this tile is
+                // issued; warp-uniform because TMEM loads and stores are warp-collective.
+                if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t ov[32];
+                        ptx::tmem_ld32(tO + 32 * c, ov);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        ptx::tmem_st32(tO + 32 * c, ov);
+                    }
+                }
+                ptx::tmem_wait_st();
+                l = l * alpha + sum;
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&p_ready[s]);
+            }
+            if (!ok) break;
+            // ------------------------------------------------------------- epilogue
+            if (!wait_warp(&o_done[s], units & 1u, sf)) break;
+            ptx::tc_fence_after();
+            const bool valid = row < p.Nq;
+            const float inv_l = 1.f / l;
+            const size_t orow = ((size_t)w.b * p.Hq + h) * (size_t)p.Nq + (size_t)(valid ? row : 0);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t ov[32];
+                ptx::tmem_ld32(tO + 32 * c, ov);
+                ptx::tmem_wait_ld();
+                if (valid) {
+                    if (OUT_F32) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
+                                                 __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                                 __uint_as_float(ov[4 * e + 2]) * inv_l,
+                                                 __uint_as_float(ov[4 * e + 3]) * inv_l);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            uint4 v4;
+                            v4.x = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
+                            v4.y = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
+                            v4.z = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
+                            v4.w = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
+                            dst[e] = v4;
+                        }
+                    }
+                }
+            }
+            if (valid) p.lse[orow] = (m + ptx::lg2(l)) * kLn2;
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&o_free[s]);
+            ++units;
+        }
+    }
+
+    __syncwarp();
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace fa

@@ -1,0 +1,204 @@
+"""ctypes binding of libfa.so (C ABI in include/fa.h) -- argument marshalling only.
+
+Every function here checks that the tensors live on a CUDA device with the expected
+dtype and contiguity, passes their device pointers and the current CUDA stream to the
+library, and raises ``FAError`` with the library's status and message on failure.  No
+attention arithmetic happens in Python; if ``libfa.so`` has not been built, every call
+raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK = 0
+FA_ERR_INVALID = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_WORKSPACE = 3
+FA_ERR_CUDA = 4
+FA_ERR_TIMEOUT = 5
+FA_ERR_DEVICE_ARG = 6
+FA_BF16 = 0
+FA_F32 = 1
+
+# Every symbol include/fa.h declares, with its ctypes signature.
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "fa_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "fa_get_error": (_I, [_P]),
+    "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
+    "fa_fwd_selftest_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_status_str": (ctypes.c_char_p, [_I]),
+    "fa_last_error_message": (ctypes.c_char_p, []),
+    "fa_version": (_I, []),
+}
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{status_str(status)}: {message}")
+
+
+def load(path: str = LIB_PATH):
+    """Load libfa.so (once) and declare its signatures.  Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise FAError(FA_ERR_UNSUPPORTED,
+                          f"{path} is not built (run: python -m exact_io_aware_81_b200.build)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_str(status: int) -> str:
+    try:
+        return load().fa_status_str(int(status)).decode()
+    except Exception:
+        return str(status)
+
+
+def _check(rc: int):
+    if rc != FA_OK:
+        raise FAError(rc, load().fa_last_error_message().decode())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {t.dim()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+        scale: Optional[float] = None, out_dtype: torch.dtype = torch.bfloat16,
+        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+        stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Attention forward: q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d) bf16 -> (o, lse).
+
+    scale defaults to 1/sqrt(d) (as flash_attn_func's softmax_scale=None does on the
+    toolsku.com page).  causal uses bottom-right alignment (row i sees keys up to
+    i + Nk - Nq).  o has out_dtype (bf16 or fp32); lse is fp32 (B,Hq,Nq), natural log.
+    """
+    _require(q, "q", torch.bfloat16, 4)
+    _require(k, "k", torch.bfloat16, 4)
+    _require(v, "v", torch.bfloat16, 4)
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, dk) != (B, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k.shape)} v {tuple(v.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=out_dtype, device=q.device)
+    else:
+        _require(out, "out", out_dtype, 4)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    else:
+        _require(lse, "lse", torch.float32, 3)
+    rc = load().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+                          FA_F32 if out_dtype == torch.float32 else FA_BF16,
+                          _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def decode_workspace_size(B: int, Hq: int, Nmax: int, d: int) -> int:
+    return int(load().fa_decode_workspace_size(B, Hq, Nmax, d))
+
+
+def decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens: torch.Tensor,
+           scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+           want_lse: bool = True, stream=None):
+    """Decode step: q (B,Hq,d) against caches (B,Hkv,Nmax,d) up to seqlens[b] (int32, device).
+
+    Returns (o (B,Hq,d) bf16, lse (B,Hq) fp32 or None).  ``workspace`` is a uint8 CUDA
+    tensor of at least decode_workspace_size(...) bytes; one is allocated if omitted.
+    """
+    _require(q, "q", torch.bfloat16, 3)
+    _require(kcache, "kcache", torch.bfloat16, 4)
+    _require(vcache, "vcache", torch.bfloat16, 4)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, d = q.shape
+    Bk, Hkv, Nmax, dk = kcache.shape
+    if (Bk, dk) != (B, d) or tuple(vcache.shape) != tuple(kcache.shape) or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, kcache, vcache and seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = decode_workspace_size(B, Hq, Nmax, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    elif not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    else:
+        _require(out, "out", torch.bfloat16, 3)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _require(lse, "lse", torch.float32, 2)
+    rc = load().fa_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
+                          out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                          B, Hq, Hkv, Nmax, d, float(scale), workspace.data_ptr(),
+                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def get_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device-side status."""
+    return int(load().fa_get_error(_stream_handle(stream)))
+
+
+def set_wait_limit_ns(ns: int):
+    load().fa_set_wait_limit_ns(int(ns))
+
+
+def fwd_selftest_timeout(q, k, v, causal=False, scale=None, stream=None):
+    """Run the prefill kernel with its score-ready signal withheld (time-limit self-test)."""
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = load().fa_fwd_selftest_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                        lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                        int(bool(causal)), _stream_handle(stream))
+    _check(rc)
+    return out, lse

@@ -1,0 +1,138 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact, IO-aware scaled-dot-product attention on B200.
+ *
+ * The operation (youngju.dev "attention variants", section 1 cost analysis and the
+ * gqa_attention example of section 2; toolsku.com generation 1 MHA formula):
+ *
+ *     O = softmax(Q K^T * scale [+ causal mask]) V,     LSE = ln sum_j exp(s_ij)
+ *
+ * computed without ever writing the (N, N) score matrix to memory: Q, K and V are
+ * staged tile by tile into on-chip memory and the softmax is accumulated online with a
+ * running row maximum and sum (youngju.dev section 3, FlashAttention).  Grouped-query
+ * sharing (youngju.dev section 2; toolsku.com generation 2): with Hq query heads and
+ * Hkv key/value heads (Hkv = G on the pages; G = Hq is MHA, G = 1 is MQA), query head h
+ * reads key/value head h / (Hq / Hkv), the repeat_interleave mapping.
+ *
+ * Conventions shared by every call
+ *   - All tensors are dense, row-major, in device memory, and owned by the caller; the
+ *     library allocates nothing per call and keeps no pointer after it returns.
+ *   - q, k, v, kcache, vcache and o must be 16-byte aligned (the TMA engine requires it).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call only
+ *     enqueues work on that stream and returns without synchronising.
+ *   - Errors in the arguments are returned synchronously and nothing is launched.
+ *     Errors the device detects (a pipeline wait that exceeded its time limit, a cache
+ *     length out of range) are recorded in a device error word that fa_get_error reads.
+ *   - Threads: the calls are thread-safe; the last error message is per host thread.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID = 1,      /* bad argument: null pointer, size <= 0, Hq % Hkv != 0,
+                                causal with Nq > Nk, scale not finite and > 0 */
+    FA_ERR_UNSUPPORTED = 2,  /* valid but not supported: d not in {64, 128}, a pointer that
+                                is not 16-byte aligned, no sm_100 device */
+    FA_ERR_WORKSPACE = 3,    /* decode workspace null or smaller than required */
+    FA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed; see fa_last_error_message */
+    FA_ERR_TIMEOUT = 5,      /* a kernel pipeline wait exceeded its time limit (fa_get_error) */
+    FA_ERR_DEVICE_ARG = 6    /* the device found seqlens[b] outside [0, Nmax] and clamped it */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
+
+/*
+ * Prefill / generic forward attention, bf16 output.
+ *   q   (B, Hq,  Nq, d) bf16          k, v (B, Hkv, Nk, d) bf16
+ *   o   (B, Hq,  Nq, d) bf16 (written)
+ *   lse (B, Hq,  Nq)    fp32 (written), natural log of sum_j exp(scale * q_i . k_j)
+ *   scale: multiplies q.k; pass 1/sqrt(d) for the usual softmax(QK^T/sqrt(d_k)).
+ *   causal != 0: row i sees keys j <= i + (Nk - Nq) (bottom-right alignment; equal to
+ *   the usual lower-triangular mask when Nq == Nk).  Requires Nq <= Nk.
+ * Supported: d in {64, 128}; any B, Hq, Hkv with Hq % Hkv == 0; any Nq, Nk >= 1.
+ */
+FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+           void *stream);
+
+/* As fa_fwd, with the output element type chosen by o_dtype (FA_BF16 or FA_F32). */
+FA_API int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+              int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+              int o_dtype, void *stream);
+
+/*
+ * Bytes of device workspace fa_decode needs for these sizes (fp32 partial outputs and
+ * partial log-sum-exps of the split-KV chunks).  0 if the sizes are invalid.
+ */
+FA_API size_t fa_decode_workspace_size(int B, int Hq, int Nmax, int d);
+
+/*
+ * Decode step over a KV cache (one query row per sequence and head): youngju.dev
+ * section 7 (decode reads the whole cache every step) and the past_kv path of the
+ * toolsku.com MHA/GQA modules (the cached keys are concatenated before the scores).
+ *   q        (B, Hq, d) bf16            kcache, vcache (B, Hkv, Nmax, d) bf16
+ *   seqlens  int32[B] in device memory, each in [0, Nmax]: sequence b attends cached
+ *            keys 0 .. seqlens[b]-1, unmasked.  seqlens[b] == 0 gives o = 0, lse = -inf.
+ *   o        (B, Hq, d) bf16 (written);  lse (B, Hq) fp32 (written) or NULL.
+ *   workspace/workspace_bytes: caller-owned device scratch of at least
+ *            fa_decode_workspace_size(B, Hq, Nmax, d) bytes, 16-byte aligned; its contents
+ *            need no initialisation and are overwritten.  Calls that share a workspace
+ *            must be ordered (same stream, or synchronised).
+ * The cache is split into chunks of 256 keys processed in parallel; the partial results
+ * are combined exactly by a log-sum-exp merge.
+ */
+FA_API int fa_decode(const void *q, const void *kcache, const void *vcache, const int *seqlens,
+              void *o, float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word.  Returns FA_OK,
+ * FA_ERR_TIMEOUT, FA_ERR_DEVICE_ARG, or FA_ERR_CUDA if the synchronisation itself failed.
+ */
+FA_API int fa_get_error(void *stream);
+
+/*
+ * Limit, in nanoseconds, on any single pipeline wait inside the kernels launched from
+ * now on by this process (default 2e9 = 2 s).  A wait that runs out records
+ * FA_ERR_TIMEOUT, makes every role of the kernel stop at its next wait, frees the
+ * kernel's tensor memory and returns.  0 restores the default.
+ */
+FA_API void fa_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Self-test of the time-limit path: launches the prefill kernel on the given (valid)
+ * arguments with its matrix-multiply warp told never to signal that a score tile is
+ * ready, so the softmax warps' first wait must run out after the wait limit.  The
+ * outputs are left unspecified; fa_get_error afterwards returns FA_ERR_TIMEOUT.
+ */
+FA_API int fa_fwd_selftest_timeout(const void *q, const void *k, const void *v, void *o, float *lse,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                            int causal, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+FA_API const char *fa_status_str(int status);
+
+/* Message of the last error returned on this host thread ("" if none). */
+FA_API const char *fa_last_error_message(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */
