@@ -320,6 +320,99 @@ int fa_decode(const void *q, const void *kcache, const void *vcache, const int *
     return ok();
 }
 
+// ------------------------------------------------------------ allocation-free decode
+//
+// For callers that cannot allocate device memory (see fa_decode_noalloc in fa.h): the
+// split-KV partials live in this fixed array instead of a caller workspace.  In host code
+// `g_noalloc_scratch` only names a host-side stand-in; its device address is looked up
+// once per device with cudaGetSymbolAddress and that address is what the kernels get.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+void *g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device (looked up on first use).
+int noalloc_scratch(int dev, void **out)
+{
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(FA_ERR_CUDA, "cudaGetSymbolAddress of the decode scratch: %s",
+                        cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return FA_OK;
+}
+
+}  // namespace
+
+int fa_decode_noalloc(const void *q, const void *kcache, const void *vcache, const int *seqlens,
+                      void *o, float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale,
+                      void *stream)
+{
+    if (!q || !kcache || !vcache || !seqlens || !o) return fail(FA_ERR_INVALID, "null pointer argument");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nmax <= 0 || d <= 0)
+        return fail(FA_ERR_INVALID, "sizes must be positive (B=%d Hq=%d Hkv=%d Nmax=%d d=%d)", B, Hq, Hkv, Nmax, d);
+    if (Hq % Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(FA_ERR_INVALID, "scale must be finite and > 0");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
+        return fail(FA_ERR_UNSUPPORTED, "q, kcache, vcache and o must be 16-byte aligned");
+    if (B > 65535 || decode_splits(Nmax) > 0x7fffffffLL)
+        return fail(FA_ERR_UNSUPPORTED, "B must be <= 65535");
+    const size_t need = decode_ws_bytes(B, Hq, Nmax, d);
+    if (need > (size_t)FA_NOALLOC_SCRATCH_BYTES)
+        return fail(FA_ERR_WORKSPACE,
+                    "this decode needs %zu bytes of scratch; fa_decode_noalloc has %u bytes "
+                    "(use fa_decode with a workspace for larger problems)",
+                    need, (unsigned)FA_NOALLOC_SCRATCH_BYTES);
+    int dev, rc;
+    DeviceInfo *info;
+    if ((rc = current_device(&dev, &info)) != FA_OK) return rc;
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(dev, &scratch)) != FA_OK) return rc;
+
+    const int R = Hq / Hkv;
+    const int rg = (R % 8 == 0) ? 8 : (R % 4 == 0) ? 4 : (R % 2 == 0) ? 2 : 1;
+    if (Hq / rg > 65535) return fail(FA_ERR_UNSUPPORTED, "too many head groups");
+
+    fa::DecodeParams p;
+    memset(&p, 0, sizeof p);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.kc = static_cast<const __nv_bfloat16 *>(kcache);
+    p.vc = static_cast<const __nv_bfloat16 *>(vcache);
+    p.seqlens = seqlens;
+    p.S_max = (int)decode_splits(Nmax);
+    p.part_o = static_cast<float *>(scratch);
+    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(scratch) +
+                                           align256((size_t)B * Hq * p.S_max * d * sizeof(float)));
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nmax = Nmax;
+    p.R = R;
+    p.scale_log2 = scale * 1.4426950408889634f;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128) launch_split_rg<128>(p, rg, st);
+    else launch_split_rg<64>(p, rg, st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
+    dim3 mgrid(Hq, B);
+    if (d == 128) fa::fa_decode_merge_kernel<128><<<mgrid, 128, 0, st>>>(p);
+    else fa::fa_decode_merge_kernel<64><<<mgrid, 128, 0, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 int fa_get_error(void *stream)
 {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -35,6 +35,7 @@ SIGNATURES = {
     "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "fa_get_error": (_I, [_P]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "fa_fwd_selftest_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
@@ -200,5 +201,39 @@ def fwd_selftest_timeout(q, k, v, causal=False, scale=None, stream=None):
     rc = load().fa_fwd_selftest_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                         lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
                                         int(bool(causal)), _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def decode_noalloc(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor,
+                   seqlens: torch.Tensor, scale: Optional[float] = None,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   stream=None):
+    """Decode step through fa_decode_noalloc: same result as ``decode`` but the library
+    uses its own fixed 32 MiB scratch instead of a workspace, for callers that cannot
+    allocate device memory.  ``out`` and ``lse`` must then be passed in by the caller;
+    calls that overlap on the GPU share the scratch and must be ordered."""
+    _require(q, "q", torch.bfloat16, 3)
+    _require(kcache, "kcache", torch.bfloat16, 4)
+    _require(vcache, "vcache", torch.bfloat16, 4)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, d = q.shape
+    Bk, Hkv, Nmax, dk = kcache.shape
+    if (Bk, dk) != (B, d) or tuple(vcache.shape) != tuple(kcache.shape) or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, kcache, vcache and seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        raise ValueError("decode_noalloc writes into a caller-provided `out`")
+    _require(out, "out", torch.bfloat16, 3)
+    if lse is not None:
+        _require(lse, "lse", torch.float32, 2)
+    rc = load().fa_decode_noalloc(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
+                                  seqlens.data_ptr(), out.data_ptr(),
+                                  lse.data_ptr() if lse is not None else None,
+                                  B, Hq, Hkv, Nmax, d, float(scale), _stream_handle(stream))
     _check(rc)
     return out, lse

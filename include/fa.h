@@ -99,6 +99,34 @@ FA_API int fa_decode(const void *q, const void *kcache, const void *vcache, cons
               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Decode step that allocates nothing and takes no workspace (no counterpart on the
+ * pages: an addition of this library for callers that cannot hand it device scratch).
+ * Some callers have no way to allocate device memory at the point of the call: plugins
+ * that only receive device pointers from a host framework that owns the allocator,
+ * serving loops that must not call cudaMalloc (it can synchronise the whole device and
+ * stall other streams), or memory pools that are fully reserved up front.  This entry
+ * point computes exactly what fa_decode computes, with the same arguments minus the
+ * workspace; its split-KV partials go to a fixed scratch array that the library keeps in
+ * device memory (FA_NOALLOC_SCRATCH_BYTES = 32 MiB on every GPU that loads libfa.so,
+ * held until the process exits).
+ *   - Limit: fa_decode_workspace_size(B, Hq, Nmax, d) must be <= FA_NOALLOC_SCRATCH_BYTES
+ *     (e.g. B * Hq * ceil(Nmax / 256) * (d + 1) * 4 bytes, each part rounded up to 256);
+ *     larger problems are rejected with FA_ERR_WORKSPACE and nothing is launched.
+ *   - The first call on each device looks up the device address of the scratch array
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any
+ *     stream capture begins.
+ *   - Every call, on every stream, shares the one scratch array and leaves its contents
+ *     behind.  Nothing in it needs to start at zero (each call writes every partial it
+ *     reads), but calls whose kernels overlap on the GPU race on it: order them (one
+ *     stream, or events) just as calls that share one fa_decode workspace.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+FA_API int fa_decode_noalloc(const void *q, const void *kcache, const void *vcache,
+                             const int *seqlens, void *o, float *lse, int B, int Hq, int Hkv,
+                             int Nmax, int d, float scale, void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word.  Returns FA_OK,
  * FA_ERR_TIMEOUT, FA_ERR_DEVICE_ARG, or FA_ERR_CUDA if the synchronisation itself failed.
  */
