@@ -152,7 +152,7 @@ int launch_prefill(const fa::PrefillParams &p, DeviceInfo *info, cudaStream_t st
             set = true;
         }
     }
-    const int grid = p.n_units < info->num_sms ? p.n_units : info->num_sms;
+    const int grid = p.n_slots < info->num_sms ? p.n_slots : info->num_sms;
     kern<<<grid, fa::prefill::kThreads, C::kSmemBytes, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(FA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
@@ -185,16 +185,18 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     p.causal = causal ? 1 : 0;
     p.head_pair = (p.R % 2 == 0) ? 1 : 0;
     const int tiles = (Nq + 127) / 128;
+    long long head_slots;
     if (p.head_pair) {
         p.T = tiles;
-        p.upt = B * Hkv * (p.R / 2);
+        head_slots = (long long)B * Hkv * (p.R / 2);
     } else {
         p.T = (tiles + 1) / 2;
-        p.upt = B * Hq;
+        head_slots = (long long)B * Hq;
     }
-    const long long units = (long long)p.T * p.upt;
-    if (units > 0x7fffffffLL) return fail(FA_ERR_UNSUPPORTED, "problem too large");
-    p.n_units = (int)units;
+    p.P = p.causal ? (p.T + 1) / 2 : p.T;
+    const long long slots = head_slots * p.P;
+    if (slots > 0x3fffffffLL) return fail(FA_ERR_UNSUPPORTED, "problem too large");
+    p.n_slots = (int)slots;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.wait_limit_ns = g_wait_limit_ns;
     p.selftest_no_s_signal = selftest_timeout;
@@ -235,6 +237,24 @@ void launch_split_rg(const fa::DecodeParams &p, int rg, cudaStream_t st)
     case 2: launch_split<D, 2>(p, st); break;
     default: launch_split<D, 1>(p, st); break;
     }
+}
+
+// The merge kernel is launched as a programmatic dependent of the split kernel, so its
+// launch overlaps the split kernel's tail; griddepcontrol.wait inside it orders the reads.
+template <int D>
+cudaError_t launch_merge(const fa::DecodeParams &p, cudaStream_t st)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.B * p.Hq));
+    cfg.blockDim = dim3(32 * fa::kMergeWarps);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fa::fa_decode_merge_kernel<D>, p);
 }
 
 }  // namespace
@@ -312,10 +332,7 @@ int fa_decode(const void *q, const void *kcache, const void *vcache, const int *
     else launch_split_rg<64>(p, rg, st);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
-    dim3 mgrid(Hq, B);
-    if (d == 128) fa::fa_decode_merge_kernel<128><<<mgrid, 128, 0, st>>>(p);
-    else fa::fa_decode_merge_kernel<64><<<mgrid, 128, 0, st>>>(p);
-    e = cudaGetLastError();
+    e = (d == 128) ? launch_merge<128>(p, st) : launch_merge<64>(p, st);
     if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -405,10 +422,7 @@ int fa_decode_noalloc(const void *q, const void *kcache, const void *vcache, con
     else launch_split_rg<64>(p, rg, st);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
-    dim3 mgrid(Hq, B);
-    if (d == 128) fa::fa_decode_merge_kernel<128><<<mgrid, 128, 0, st>>>(p);
-    else fa::fa_decode_merge_kernel<64><<<mgrid, 128, 0, st>>>(p);
-    e = cudaGetLastError();
+    e = (d == 128) ? launch_merge<128>(p, st) : launch_merge<64>(p, st);
     if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
     return ok();
 }

@@ -62,6 +62,61 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8])
     }
 }
 
+__device__ __forceinline__ void unpack8x2(const uint4 &u, float2 (&f)[4])
+{
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+
+// Sums V values per lane over the LPK lanes that share one key row and scatters the
+// results: after the call lane `sub` holds, in a[0], the full sum of value head_of(sub).
+// Levels with more than one value left halve the values (a lane keeps one half and adds
+// its partner's copy of that half), the remaining levels are plain butterflies.
+template <int V, int LPK>
+__device__ __forceinline__ void reduce_scatter(float (&a)[V], int sub)
+{
+    int n = V;
+#pragma unroll
+    for (int off = LPK / 2; off >= 1; off >>= 1) {
+        if (n > 1) {
+            const int half = n >> 1;
+            const bool upper = (sub & off) != 0;
+#pragma unroll
+            for (int i = 0; i < V / 2; ++i) {
+                if (i < half) {
+                    const float send = upper ? a[i] : a[i + half];
+                    const float keep = upper ? a[i + half] : a[i];
+                    a[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
+            }
+            n = half;
+        } else {
+            a[0] += __shfl_xor_sync(0xffffffffu, a[0], off);
+        }
+    }
+}
+
+// Which value lane `sub` holds after reduce_scatter<V, LPK>, and whether it is the one
+// lane (of the group holding that value) that writes it.
+template <int V, int LPK>
+__device__ __forceinline__ int scatter_head(int sub, bool &writer)
+{
+    int head = 0, n = V, low_mask = 0;
+#pragma unroll
+    for (int off = LPK / 2; off >= 1; off >>= 1) {
+        if (n > 1) {
+            n >>= 1;
+            if (sub & off) head += n;
+        } else {
+            low_mask |= off;
+        }
+    }
+    writer = (sub & low_mask) == 0;
+    return head;
+}
+
 __device__ __forceinline__ uint4 ldg_stream(const void *p)
 {
     uint4 r;
@@ -87,6 +142,9 @@ __global__ void __launch_bounds__(decode::kThreads)
     __shared__ float red[kWarps][RG][D];
     __shared__ float m_sm[RG], l_sm[RG];
 
+    // let the merge kernel (launched as a programmatic dependent) get scheduled early; it
+    // waits for this whole grid to finish before it reads any partial
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int chunk = blockIdx.x;
     const int h0 = blockIdx.y * RG;
     const int b = blockIdx.z;
@@ -107,14 +165,16 @@ __global__ void __launch_bounds__(decode::kThreads)
     const __nv_bfloat16 *kbase = p.kc + plane * D + sub * 8;
     const __nv_bfloat16 *vbase = p.vc + plane * D + sub * 8;
 
-    float qf[RG][8];
+    float2 qf[RG][4];
 #pragma unroll
     for (int r = 0; r < RG; ++r) {
         const uint4 u = *reinterpret_cast<const uint4 *>(p.q + ((size_t)b * p.Hq + h0 + r) * D + sub * 8);
-        unpack8(u, qf[r]);
+        unpack8x2(u, qf[r]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) qf[r][e] *= p.scale_log2;
+        for (int e = 0; e < 4; ++e) qf[r][e] = __fmul2_rn(qf[r][e], make_float2(p.scale_log2, p.scale_log2));
     }
+    bool writer;
+    const int my_head = scatter_head<RG, LPK>(sub, writer);
 
     // ---------------------------------------------------------------- K pass
     for (int base = 0; base < n; base += KPI * kUnroll) {
@@ -127,24 +187,18 @@ __global__ void __launch_bounds__(decode::kThreads)
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int key = base + u * KPI + warp * KPW + kk;
-            float kf[8];
-            unpack8(kr[u], kf);
+            float2 kf[4];
+            unpack8x2(kr[u], kf);
             float acc[RG];
 #pragma unroll
             for (int r = 0; r < RG; ++r) {
-                float a = 0.f;
+                float2 a = __fmul2_rn(qf[r][0], kf[0]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) a = fmaf(qf[r][e], kf[e], a);
-                acc[r] = a;
+                for (int e = 1; e < 4; ++e) a = __ffma2_rn(qf[r][e], kf[e], a);
+                acc[r] = a.x + a.y;
             }
-#pragma unroll
-            for (int off = 1; off < LPK; off <<= 1)
-#pragma unroll
-                for (int r = 0; r < RG; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], off);
-            if (sub == 0 && key < n) {
-#pragma unroll
-                for (int r = 0; r < RG; ++r) s_sm[r][key] = acc[r];
-            }
+            reduce_scatter<RG, LPK>(acc, sub);
+            if (writer && key < n) s_sm[my_head][key] = acc[0];
         }
     }
     __syncthreads();
@@ -171,11 +225,11 @@ __global__ void __launch_bounds__(decode::kThreads)
     __syncthreads();
 
     // ---------------------------------------------------------------- V pass
-    float acc[RG][8];
+    float2 acc[RG][4];
 #pragma unroll
     for (int r = 0; r < RG; ++r)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
+        for (int e = 0; e < 4; ++e) acc[r][e] = make_float2(0.f, 0.f);
     for (int base = 0; base < n; base += KPI * kUnroll) {
         uint4 vr[kUnroll];
 #pragma unroll
@@ -187,13 +241,14 @@ __global__ void __launch_bounds__(decode::kThreads)
         for (int u = 0; u < kUnroll; ++u) {
             const int key = base + u * KPI + warp * KPW + kk;
             if (key < n) {
-                float vf[8];
-                unpack8(vr[u], vf);
+                float2 vf[4];
+                unpack8x2(vr[u], vf);
 #pragma unroll
                 for (int r = 0; r < RG; ++r) {
                     const float pr = s_sm[r][key];
+                    const float2 p2 = make_float2(pr, pr);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(pr, vf[e], acc[r][e]);
+                    for (int e = 0; e < 4; ++e) acc[r][e] = __ffma2_rn(p2, vf[e], acc[r][e]);
                 }
             }
         }
@@ -204,12 +259,18 @@ __global__ void __launch_bounds__(decode::kThreads)
 #pragma unroll
         for (int r = 0; r < RG; ++r)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[r][e] += __shfl_xor_sync(0xffffffffu, acc[r][e], off);
+            for (int e = 0; e < 4; ++e) {
+                acc[r][e].x += __shfl_xor_sync(0xffffffffu, acc[r][e].x, off);
+                acc[r][e].y += __shfl_xor_sync(0xffffffffu, acc[r][e].y, off);
+            }
     if (kk == 0) {
 #pragma unroll
         for (int r = 0; r < RG; ++r)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) red[warp][r][sub * 8 + e] = acc[r][e];
+            for (int e = 0; e < 4; ++e) {
+                red[warp][r][sub * 8 + 2 * e] = acc[r][e].x;
+                red[warp][r][sub * 8 + 2 * e + 1] = acc[r][e].y;
+            }
     }
     __syncthreads();
 
@@ -226,16 +287,28 @@ __global__ void __launch_bounds__(decode::kThreads)
             m_sm[threadIdx.x] + ptx::lg2(l_sm[threadIdx.x]);
 }
 
-// One CTA per (query head, sequence); thread e owns output element e.
+// One CTA of kMergeWarps warps per (query head, sequence).  Every warp finds the largest
+// partial log2-sum-exp M (lanes stride over the S partials); warp w then accumulates the
+// weighted partial outputs of splits w, w + kMergeWarps, ... with each lane owning D/32
+// consecutive elements; the warps' sums are added in shared memory.
+constexpr int kMergeWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(128) fa_decode_merge_kernel(const __grid_constant__ DecodeParams p)
+__global__ void __launch_bounds__(32 * kMergeWarps) fa_decode_merge_kernel(const __grid_constant__ DecodeParams p)
 {
     using namespace decode;
-    const int h = blockIdx.x;
-    const int b = blockIdx.y;
+    // wait until the split kernel's partials are complete and visible (no-op when this
+    // kernel was not launched as a programmatic dependent)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    constexpr int EPL = D / 32;  // output elements per lane
+    __shared__ float red[kMergeWarps][D];
+    __shared__ float den_sm[kMergeWarps];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const size_t bh = blockIdx.x;
+    const int b = (int)(bh / p.Hq);
     const int L = clamp_len(p.seqlens[b], p.Nmax);
     const int S = (L + kChunk - 1) / kChunk;
-    const size_t bh = (size_t)b * p.Hq + h;
     const float *pl = p.part_lse + bh * p.S_max;
     const float *po = p.part_o + bh * p.S_max * D;
     if (S == 0) {
@@ -244,16 +317,35 @@ __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const __grid_const
         return;
     }
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, pl[s]);
-    float den = 0.f, num = 0.f;
-    const int e = threadIdx.x;
-    for (int s = 0; s < S; ++s) {
+    for (int s = lane; s < S; s += 32) M = fmaxf(M, pl[s]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float den = 0.f;
+    float acc[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+#pragma unroll 4
+    for (int s = warp; s < S; s += kMergeWarps) {
         const float w = ptx::ex2(pl[s] - M);
         den += w;
-        if (e < D) num = fmaf(w, po[(size_t)s * D + e], num);
+        const float *src = po + (size_t)s * D + lane * EPL;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, src[e], acc[e]);
     }
-    if (e < D) p.o[bh * D + e] = __float2bfloat16_rn(num / den);
-    if (e == 0 && p.lse) p.lse[bh] = (M + ptx::lg2(den)) * kLn2;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) red[warp][lane * EPL + e] = acc[e];
+    if (lane == 0) den_sm[warp] = den;
+    __syncthreads();
+    if (threadIdx.x < D) {
+        float t = 0.f, dsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMergeWarps; ++w) {
+            t += red[w][threadIdx.x];
+            dsum += den_sm[w];
+        }
+        p.o[bh * D + threadIdx.x] = __float2bfloat16_rn(t / dsum);
+        if (threadIdx.x == 0 && p.lse) p.lse[bh] = (M + ptx::lg2(dsum)) * kLn2;
+    }
 }
 
 }  // namespace fa

@@ -12,8 +12,10 @@
 //
 // B200 mapping (one persistent CTA per SM, 12 warps = 3 warpgroups):
 //   warp 8      TMA producer: Q tiles once per work unit, K_j / V_j into an NSTAGE ring
-//               of 128-byte-swizzled tiles, completion counted on mbarriers.
-//   warp 9      MMA issuer: S_s = Q_s K_j^T (both operands from shared memory) and
+//               of 128-byte-swizzled tiles, completion counted on mbarriers (the warp
+//               runs the loop, one elected lane issues).
+//   warp 9      MMA issuer (warp runs the loop, one elected lane issues):
+//               S_s = Q_s K_j^T (both operands from shared memory) and
 //               O_s += P_s V_j (P from tensor memory, V from shared memory) with
 //               tcgen05.mma; accumulators live in tensor memory (512 columns:
 //               S0 | S1 | O0 | O1, P_s packed as bf16 over the first 64 columns of S_s).
@@ -23,7 +25,8 @@
 //               moved when the new one exceeds it by more than 8 in log2 units; O_s is
 //               then rescaled in TMEM by the same warp), P_s to TMEM as bf16, fp32 row
 //               sum; at the end of a unit O_s / l and LSE are written out.
-//   warps 10-11 idle (they complete the third warpgroup).
+//   warps 10-11 idle (they complete the third warpgroup, which lends registers to the
+//               softmax warpgroups through setmaxnreg).
 // The two Q tiles of a work unit share their key/value head: two query heads of one
 // group (R even) or two consecutive row tiles of one head (otherwise).  Their MMAs are
 // interleaved S0_j, PV1_{j-1}, S1_j, PV0_j so that the tensor core works on one tile
@@ -49,9 +52,9 @@ struct PrefillParams {
     int R;           // Hq / Hkv
     int causal;
     int head_pair;   // 1: a unit = heads (2p, 2p+1) of one group on the same 128 rows
-    int n_units;
-    int T;           // tile rows: 128-row tiles (head_pair) or 256-row tile pairs
-    int upt;         // units per tile row
+    int T;           // tile rows per head slot: 128-row tiles (head_pair) or 256-row pairs
+    int P;           // slots per head slot: ceil(T/2) if causal (units paired), else T
+    int n_slots;     // head slots * P
     float scale_log2;  // scale * log2(e)
     unsigned long long wait_limit_ns;
     int selftest_no_s_signal;  // timeout self-test: never signal a ready score tile
@@ -62,6 +65,12 @@ namespace prefill {
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int kThreads = 384;   // 3 warpgroups
+// Registers per thread: 168 at launch (384 threads share the 64K register file).  With
+// setmaxnreg the producer/MMA warpgroup keeps kRegsLow and each softmax warpgroup gets
+// kRegsHigh; 128 * kRegsLow + 256 * kRegsHigh must not exceed 384 * 168.
+constexpr int kRegsLow = 72;
+constexpr int kRegsHigh = 216;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch budget");
 constexpr int kChunkBytes = 128 * 128;  // one 64-column (128-byte) slab of a 128-row tile
 constexpr float kLazyThreshold = 8.0f;  // log2 units: rescale only past a factor of 256
 constexpr float kLn2 = 0.6931471805599453f;
@@ -84,24 +93,35 @@ struct Unit {
     int b, g, h0, h1, r0, r1, n0, n1;
 };
 
-__device__ __forceinline__ Unit decode_unit(const PrefillParams &p, int u)
+// Work is dealt out in slots.  A slot belongs to one "head slot" (a head pair of one
+// K/V group, or one head) and, for causal masks, holds two units: tile row T-1-i (the
+// heaviest left) and tile row i (the lightest), so every slot costs the same and a plain
+// round-robin over the persistent CTAs stays balanced.  Head slots are numbered with the
+// heads of one K/V group adjacent and slots of one head slot consecutive, so the CTAs
+// running at any moment share few K/V heads and their tiles are re-read from L2.
+__device__ __forceinline__ int units_in_slot(const PrefillParams &p) { return p.causal ? 2 : 1; }
+
+__device__ __forceinline__ bool decode_unit(const PrefillParams &p, int slot, int k, Unit &w)
 {
-    Unit w;
-    const int tr = u / p.upt;
-    const int rem = u - tr * p.upt;
-    const int t = p.causal ? (p.T - 1 - tr) : tr;  // causal: heaviest tile rows first
+    const int hh = slot / p.P;
+    const int pi = slot - hh * p.P;
+    int t = pi;
+    if (p.causal) {
+        t = (k == 0) ? (p.T - 1 - pi) : pi;
+        if (k == 1 && pi == p.T - 1 - pi) return false;  // middle tile row of an odd T
+    }
     if (p.head_pair) {
         const int hpairs = p.R >> 1;
-        const int hp = rem % hpairs;
-        const int bg = rem / hpairs;
+        const int hp = hh % hpairs;
+        const int bg = hh / hpairs;
         w.g = bg % p.Hkv;
         w.b = bg / p.Hkv;
         w.h0 = w.g * p.R + 2 * hp;
         w.h1 = w.h0 + 1;
         w.r0 = w.r1 = BM * t;
     } else {
-        const int h = rem % p.Hq;
-        w.b = rem / p.Hq;
+        const int h = hh % p.Hq;
+        w.b = hh / p.Hq;
         w.g = h / p.R;
         w.h0 = w.h1 = h;
         w.r0 = 2 * BM * t;
@@ -116,7 +136,7 @@ __device__ __forceinline__ Unit decode_unit(const PrefillParams &p, int u)
     } else {
         w.n0 = w.n1 = nkt;
     }
-    return w;
+    return true;
 }
 
 // S = Q K^T over the full head dimension: D/16 MMAs of K = 16.  Both operands are
@@ -149,6 +169,71 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
     for (int k = 0; k < BN / 16; ++k) {
         const uint64_t b = ptx::smem_desc_sw128(v_saddr + k * 2048, kChunkBytes, 1024);
         ptx::mma_ts(d_tmem, p_tmem + k * 8, b, idesc, (accumulate || k > 0) ? 1u : 0u);
+    }
+}
+
+// Pairs of exponentials evaluated on the FMA pipe (exp2_poly2) instead of the MUFU unit:
+// pair c does when kPolyPeriod > 0 and c % kPolyPeriod == kPolyPeriod - 1.  Measured on
+// B200 with this kernel, moving 1/4, 3/8 or 1/2 of them to the FMA pipe made it slower
+// (the softmax is not MUFU-throughput bound here), so the offload is off.
+constexpr int kPolyPeriod = 0;
+
+// p = 2^(x * sl2 - m) for NC scores of a row held as raw fp32 bits in x[IN .. IN+NC); the
+// p are packed as bf16 pairs into x[OUT .. OUT+NC/2) (OUT <= IN, so every score is read
+// before its slot is overwritten) and their fp32 sum is returned.  Lane pairs use packed
+// fp32x2 math.
+template <int NC, int IN, int OUT>
+__device__ __forceinline__ float exp2_pack(uint32_t (&x)[128], float sl2, float m)
+{
+    static_assert(OUT <= IN && NC % 8 == 0, "in-place packing order");
+    const float2 c2 = make_float2(sl2, sl2);
+    const float2 nm2 = make_float2(-m, -m);
+    float2 acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < NC / 2; ++c) {
+        const float2 y = __ffma2_rn(make_float2(__uint_as_float(x[IN + 2 * c]), __uint_as_float(x[IN + 2 * c + 1])), c2, nm2);
+        float2 e;
+        if (kPolyPeriod > 0 && c % kPolyPeriod == kPolyPeriod - 1) {
+            e = ptx::exp2_poly2(y);
+        } else {
+            e.x = ptx::ex2(y.x);
+            e.y = ptx::ex2(y.y);
+        }
+        acc[c & 3] = __fadd2_rn(acc[c & 3], e);
+        x[OUT + c] = ptx::pack_bf16x2(e.x, e.y);
+    }
+    const float2 s01 = __fadd2_rn(acc[0], acc[1]);
+    const float2 s23 = __fadd2_rn(acc[2], acc[3]);
+    const float2 t = __fadd2_rn(s01, s23);
+    return t.x + t.y;
+}
+
+// Maximum of 64 scores x[IN .. IN+64) (four chains of three-input max).
+template <int IN>
+__device__ __forceinline__ float row_max64(const uint32_t (&x)[128])
+{
+    float a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t *v = &x[IN + 16 * i];
+        float t = ptx::max3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+        for (int k = 3; k < 15; k += 2) t = ptx::max3(t, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
+        a[i] = fmaxf(t, __uint_as_float(v[15]));
+    }
+    return fmaxf(ptx::max3(a[0], a[1], a[2]), a[3]);
+}
+
+// Set scores of keys past this row's last visible key to -inf (columns [C0, C0+NC)).
+template <int C0, int NC>
+__device__ __forceinline__ void mask_cols(uint32_t (&x)[128], int kbase, int lim)
+{
+    if (kbase + C0 + NC - 1 > lim) {
+#pragma unroll
+        for (int c = C0; c < C0 + NC; ++c)
+            if (kbase + c > lim) x[c] = __float_as_uint(-INFINITY);
     }
 }
 
@@ -231,16 +316,21 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
 
     if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            uint32_t kv_it = 0, q_it = 0;
-            uint32_t q_fills[2] = {0u, 0u};
-            bool ok = true;
-            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
-                const Unit w = decode_unit(p, u);
-                for (int s = 0; s < 2 && ok; ++s) {
-                    if (!wait_one(&q_empty[s], (q_it & 1u) ^ 1u, sf)) { ok = false; break; }
+        // The whole warp runs the loop (every value is warp-uniform); one elected lane
+        // issues the copies.
+        ptx::regs_decrease<kRegsLow>();
+        const bool leader = ptx::elect_one();
+        uint32_t kv_it = 0, q_it = 0;
+        uint32_t q_fills[2] = {0u, 0u};
+        bool ok = true;
+        for (int u = blockIdx.x * 2; ok && u < p.n_slots * 2; u += (u & 1) ? 2 * gridDim.x - 1 : 1) {
+            Unit w;
+            if ((u & 1) >= units_in_slot(p) || !decode_unit(p, u >> 1, u & 1, w)) continue;
+            for (int s = 0; s < 2 && ok; ++s) {
+                if (!wait_warp(&q_empty[s], (q_it & 1u) ^ 1u, sf)) { ok = false; break; }
+                ++q_fills[s];
+                if (leader) {
                     ptx::mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
-                    ++q_fills[s];
                     const int h = s ? w.h1 : w.h0;
                     const int r = s ? w.r1 : w.r0;
                     uint8_t *dst = smem + C::kQOff + s * C::kTileBytes;
@@ -249,14 +339,17 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                         ptx::tma_load_3d(dst + c * kChunkBytes, &p.tm_q, &q_full[s], 64 * c, r,
                                          w.b * p.Hq + h);
                 }
-                if (!ok) break;
-                ++q_it;
-                const int plane = w.b * p.Hkv + w.g;
-                for (int j = 0; j < w.n1 && ok; ++j) {
-                    for (int kv = 0; kv < 2; ++kv) {
-                        const uint32_t st = kv_it % C::kStages;
-                        const uint32_t ph = (kv_it / C::kStages) & 1u;
-                        if (!wait_one(&kv_empty[st], ph ^ 1u, sf)) { ok = false; break; }
+                __syncwarp();
+            }
+            if (!ok) break;
+            ++q_it;
+            const int plane = w.b * p.Hkv + w.g;
+            for (int j = 0; j < w.n1 && ok; ++j) {
+                for (int kv = 0; kv < 2; ++kv) {
+                    const uint32_t st = kv_it % C::kStages;
+                    const uint32_t ph = (kv_it / C::kStages) & 1u;
+                    if (!wait_warp(&kv_empty[st], ph ^ 1u, sf)) { ok = false; break; }
+                    if (leader) {
                         ptx::mbar_arrive_expect_tx(&kv_full[st], C::kTileBytes);
                         uint8_t *dst = smem + C::kKVOff + st * C::kTileBytes;
                         const CUtensorMap *map = kv ? &p.tm_v : &p.tm_k;
@@ -264,11 +357,14 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                         for (int c = 0; c < D / 64; ++c)
                             ptx::tma_load_3d(dst + c * kChunkBytes, map, &kv_full[st], 64 * c,
                                              BN * j, plane);
-                        ++kv_it;
                     }
+                    __syncwarp();
+                    ++kv_it;
                 }
             }
-            // Let every copy this thread started land before the CTA can exit.
+        }
+        // Let every copy this warp started land before the CTA can exit.
+        if (leader) {
             for (uint32_t st = 0; st < (uint32_t)C::kStages && st < kv_it; ++st) {
                 const uint32_t last = kv_it - 1 - ((kv_it - 1 - st) % C::kStages);
                 drain_wait(&kv_full[st], (last / C::kStages) & 1u, p.wait_limit_ns);
@@ -276,73 +372,97 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             for (int s = 0; s < 2; ++s)
                 if (q_fills[s] > 0) drain_wait(&q_full[s], (q_fills[s] - 1) & 1u, p.wait_limit_ns);
         }
+        __syncwarp();
     } else if (warp == 9) {
         // --------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            uint32_t kv_it = 0, units = 0;
-            uint32_t p_ph[2] = {0u, 0u};
-            bool ok = true;
-            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
-                const Unit w = decode_unit(p, u);
-                const uint32_t q_par = units & 1u;
-                const uint32_t free_par = q_par ^ 1u;  // first unit passes at once
-                if (!wait_one(&q_full[0], q_par, sf) || !wait_one(&q_full[1], q_par, sf)) break;
+        // The whole warp runs the loop, so descriptors and addresses are warp-uniform;
+        // one elected lane issues each group of MMAs and its commits.
+        ptx::regs_decrease<kRegsLow>();
+        const bool leader = ptx::elect_one();
+        const bool signal_s = !p.selftest_no_s_signal;
+        uint32_t kv_it = 0, units = 0;
+        uint32_t p_ph[2] = {0u, 0u};
+        bool ok = true;
+        for (int u = blockIdx.x * 2; ok && u < p.n_slots * 2; u += (u & 1) ? 2 * gridDim.x - 1 : 1) {
+            Unit w;
+            if ((u & 1) >= units_in_slot(p) || !decode_unit(p, u >> 1, u & 1, w)) continue;
+            const uint32_t q_par = units & 1u;
+            const uint32_t free_par = q_par ^ 1u;  // first unit passes at once
+            if (!wait_warp(&q_full[0], q_par, sf) || !wait_warp(&q_full[1], q_par, sf)) break;
+            ptx::tc_fence_after();
+            uint32_t prev_v = 0;
+            for (int j = 0; j < w.n1; ++j) {
+                const uint32_t ks = kv_it % C::kStages;
+                const uint32_t kph = (kv_it / C::kStages) & 1u;
+                const uint32_t vs = (kv_it + 1) % C::kStages;
+                const uint32_t vph = ((kv_it + 1) / C::kStages) & 1u;
+                if (!wait_warp(&kv_full[ks], kph, sf)) { ok = false; break; }
                 ptx::tc_fence_after();
-                uint32_t prev_v = 0;
-                for (int j = 0; j < w.n1; ++j) {
-                    const uint32_t ks = kv_it % C::kStages;
-                    const uint32_t kph = (kv_it / C::kStages) & 1u;
-                    const uint32_t vs = (kv_it + 1) % C::kStages;
-                    const uint32_t vph = ((kv_it + 1) / C::kStages) & 1u;
-                    if (!wait_one(&kv_full[ks], kph, sf)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t k_saddr = kv_saddr0 + ks * C::kTileBytes;
-                    if (j < w.n0) {
+                const uint32_t k_saddr = kv_saddr0 + ks * C::kTileBytes;
+                if (j < w.n0) {
+                    if (leader) {
                         issue_qk<D>(tmem + 0, q_saddr0, k_saddr);
-                        if (!p.selftest_no_s_signal) ptx::mma_commit(&s_full[0]);
+                        if (signal_s) ptx::mma_commit(&s_full[0]);
                         if (j == w.n0 - 1) ptx::mma_commit(&q_empty[0]);
                     }
-                    if (j > 0) {
-                        if (!wait_one(&p_ready[1], p_ph[1], sf)) { ok = false; break; }
-                        p_ph[1] ^= 1u;
-                        if (j - 1 == 0 && !wait_one(&o_free[1], free_par, sf)) { ok = false; break; }
-                        ptx::tc_fence_after();
+                    __syncwarp();
+                }
+                if (j > 0) {
+                    if (!wait_warp(&p_ready[1], p_ph[1], sf)) { ok = false; break; }
+                    p_ph[1] ^= 1u;
+                    if (j - 1 == 0 && !wait_warp(&o_free[1], free_par, sf)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    if (leader) {
                         issue_pv<D>(tmem + 384, tmem + 128, kv_saddr0 + prev_v * C::kTileBytes, j - 1 > 0);
                         ptx::mma_commit(&kv_empty[prev_v]);
                     }
+                    __syncwarp();
+                }
+                if (leader) {
                     issue_qk<D>(tmem + 128, q_saddr0 + C::kTileBytes, k_saddr);
-                    if (!p.selftest_no_s_signal) ptx::mma_commit(&s_full[1]);
+                    if (signal_s) ptx::mma_commit(&s_full[1]);
                     ptx::mma_commit(&kv_empty[ks]);
                     if (j == w.n1 - 1) ptx::mma_commit(&q_empty[1]);
-                    if (!wait_one(&kv_full[vs], vph, sf)) { ok = false; break; }
-                    if (j < w.n0) {
-                        if (!wait_one(&p_ready[0], p_ph[0], sf)) { ok = false; break; }
-                        p_ph[0] ^= 1u;
-                        if (j == 0 && !wait_one(&o_free[0], free_par, sf)) { ok = false; break; }
-                        ptx::tc_fence_after();
+                }
+                __syncwarp();
+                if (!wait_warp(&kv_full[vs], vph, sf)) { ok = false; break; }
+                if (j < w.n0) {
+                    if (!wait_warp(&p_ready[0], p_ph[0], sf)) { ok = false; break; }
+                    p_ph[0] ^= 1u;
+                    if (j == 0 && !wait_warp(&o_free[0], free_par, sf)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    if (leader) {
                         issue_pv<D>(tmem + 256, tmem + 0, kv_saddr0 + vs * C::kTileBytes, j > 0);
                         if (j == w.n0 - 1) ptx::mma_commit(&o_done[0]);
                     }
-                    prev_v = vs;
-                    kv_it += 2;
+                    __syncwarp();
                 }
-                if (!ok) break;
-                // last P V of tile 1
-                if (!wait_one(&p_ready[1], p_ph[1], sf)) break;
-                p_ph[1] ^= 1u;
-                if (w.n1 == 1 && !wait_one(&o_free[1], free_par, sf)) break;
-                ptx::tc_fence_after();
+                prev_v = vs;
+                kv_it += 2;
+            }
+            if (!ok) break;
+            // last P V of tile 1
+            if (!wait_warp(&p_ready[1], p_ph[1], sf)) break;
+            p_ph[1] ^= 1u;
+            if (w.n1 == 1 && !wait_warp(&o_free[1], free_par, sf)) break;
+            ptx::tc_fence_after();
+            if (leader) {
                 issue_pv<D>(tmem + 384, tmem + 128, kv_saddr0 + prev_v * C::kTileBytes, w.n1 > 1);
                 ptx::mma_commit(&kv_empty[prev_v]);
                 ptx::mma_commit(&o_done[1]);
-                ++units;
             }
-            // Every MMA and commit issued above completes before the CTA can exit.
+            __syncwarp();
+            ++units;
+        }
+        // Every MMA and commit issued above completes before the CTA can exit.
+        if (leader) {
             ptx::mma_commit(teardown);
             drain_wait(teardown, 0, p.wait_limit_ns);
         }
+        __syncwarp();
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax warps
+        ptx::regs_increase<kRegsHigh>();
         const int s = warp >> 2;              // which Q tile of the unit
         const int tid = threadIdx.x & 127;    // row inside the tile = TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -350,54 +470,46 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         const uint32_t tO = tmem + lane_base + 256u + 128u * s;  // O_s
         const float sl2 = p.scale_log2;
         uint32_t s_ph = 0, units = 0;
-        for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-            const Unit w = decode_unit(p, u);
+        for (int u = blockIdx.x * 2; u < p.n_slots * 2; u += (u & 1) ? 2 * gridDim.x - 1 : 1) {
+            Unit w;
+            if ((u & 1) >= units_in_slot(p) || !decode_unit(p, u >> 1, u & 1, w)) continue;
             const int h = s ? w.h1 : w.h0;
             const int r0 = s ? w.r1 : w.r0;
             const int n = s ? w.n1 : w.n0;
             const int row = r0 + tid;
             const int lim = p.causal ? min(row + (p.Nk - p.Nq), p.Nk - 1) : p.Nk - 1;
-            float m = -INFINITY, l = 0.f;
+            // l: sum of the fp32 weights (gives the LSE).  lo: normaliser of O, the same sum
+            // corrected, tile by tile, by the bf16 rounding of the tile's largest weight --
+            // the rounding the P V product actually saw.  For a row dominated by one key
+            // this makes O exactly that key's value row, as it should be.
+            float m = -INFINITY, l = 0.f, lo = 0.f;
             bool ok = true;
             for (int j = 0; j < n; ++j) {
                 if (!wait_warp(&s_full[s], s_ph, sf)) { ok = false; break; }
                 s_ph ^= 1u;
                 ptx::tc_fence_after();
                 uint32_t x[128];
+                const int kbase = BN * j;
+                float alpha = 1.f, sum, mx;
+                bool rescale = false;
+                // Scores of this tile, masked past the row's last visible key; the tile
+                // maximum; lazy update of the reference maximum m (moved only when the new
+                // one exceeds it by more than kLazyThreshold, which then rescales O).
                 ptx::tmem_ld32(tS + 0, &x[0]);
                 ptx::tmem_ld32(tS + 32, &x[32]);
                 ptx::tmem_ld32(tS + 64, &x[64]);
                 ptx::tmem_ld32(tS + 96, &x[96]);
                 ptx::tmem_wait_ld();
-                const int kbase = BN * j;
-                if (kbase + BN - 1 > lim) {
-#pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (kbase + c > lim) x[c] = __float_as_uint(-INFINITY);
-                }
-                float mx = __uint_as_float(x[0]);
-#pragma unroll
-                for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(x[c]));
-                const float m_new = fmaxf(m, mx * sl2);
-                float alpha = 1.f;
-                bool rescale = false;
+                mask_cols<0, 128>(x, kbase, lim);
+                mx = fmaxf(row_max64<0>(x), row_max64<64>(x)) * sl2;
                 if (j == 0) {
-                    m = m_new;
-                } else if (m_new - m > kLazyThreshold) {
-                    alpha = ptx::ex2(m - m_new);
-                    m = m_new;
+                    m = mx;  // O is not written yet: the first P V overwrites it
+                } else if (mx - m > kLazyThreshold) {
+                    alpha = ptx::ex2(m - mx);
+                    m = mx;
                     rescale = true;
                 }
-                // P = 2^(s * scale * log2e - m), packed in place as bf16 pairs.
-                const float negm = -m;
-                float sum = 0.f;
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float p0 = ptx::ex2(fmaf(__uint_as_float(x[2 * c]), sl2, negm));
-                    const float p1 = ptx::ex2(fmaf(__uint_as_float(x[2 * c + 1]), sl2, negm));
-                    sum += p0 + p1;
-                    x[c] = ptx::pack_bf16x2(p0, p1);
-                }
+                sum = exp2_pack<64, 0, 0>(x, sl2, m) + exp2_pack<64, 64, 32>(x, sl2, m);
                 ptx::tmem_st32(tS + 0, &x[0]);
                 ptx::tmem_st32(tS + 32, &x[32]);
                 // Rare (lazy) rescale of the partial output, before P V of this tile is
@@ -415,7 +527,10 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     }
                 }
                 ptx::tmem_wait_st();
+                const float p_top = ptx::ex2(mx - m);  // the tile's largest weight (0 if masked)
+                const float p_top_bf = __uint_as_float(ptx::pack_bf16x2(p_top, 0.f) << 16);
                 l = l * alpha + sum;
+                lo = lo * alpha + sum + (p_top_bf - p_top);
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&p_ready[s]);
             }
@@ -424,33 +539,31 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             if (!wait_warp(&o_done[s], units & 1u, sf)) break;
             ptx::tc_fence_after();
             const bool valid = row < p.Nq;
-            const float inv_l = 1.f / l;
+            const float inv_l = 1.f / lo;
             const size_t orow = ((size_t)w.b * p.Hq + h) * (size_t)p.Nq + (size_t)(valid ? row : 0);
+            uint32_t ov[D];
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t ov[32];
-                ptx::tmem_ld32(tO + 32 * c, ov);
-                ptx::tmem_wait_ld();
-                if (valid) {
-                    if (OUT_F32) {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D + 32 * c);
+            for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(tO + 32 * c, &ov[32 * c]);
+            ptx::tmem_wait_ld();
+            if (valid) {
+                if (OUT_F32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
-                                                 __uint_as_float(ov[4 * e + 1]) * inv_l,
-                                                 __uint_as_float(ov[4 * e + 2]) * inv_l,
-                                                 __uint_as_float(ov[4 * e + 3]) * inv_l);
-                    } else {
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D + 32 * c);
+                    for (int e = 0; e < D / 4; ++e)
+                        dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
+                                             __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                             __uint_as_float(ov[4 * e + 2]) * inv_l,
+                                             __uint_as_float(ov[4 * e + 3]) * inv_l);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            uint4 v4;
-                            v4.x = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
-                            v4.y = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
-                            v4.z = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
-                            v4.w = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
-                            dst[e] = v4;
-                        }
+                    for (int e = 0; e < D / 8; ++e) {
+                        uint4 v4;
+                        v4.x = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
+                        v4.y = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
+                        v4.z = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
+                        v4.w = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
+                        dst[e] = v4;
                     }
                 }
             }
@@ -461,6 +574,9 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         }
     }
 
+    else {
+        ptx::regs_decrease<kRegsLow>();
+    }
     __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();

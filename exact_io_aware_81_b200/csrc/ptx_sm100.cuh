@@ -175,6 +175,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
         : "memory");
 }
 
+// True in exactly one lane of a fully active warp.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Register re-balancing between warpgroups (whole warpgroup, count multiple of 8).
 template <int N>
 __device__ __forceinline__ void regs_increase() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
@@ -221,6 +233,36 @@ __device__ __forceinline__ float lg2(float x)
     float y;
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^y for two lanes on the FMA pipe, for y <= 2^22 (masked -inf included): y is clamped to
+// >= -127, split as y = j + f with j = round(y) (by adding and subtracting 1.5 * 2^23) and
+// f in [-1/2, 1/2]; q(f) ~ 2^f is a degree-3 polynomial with q(0) = 1 whose coefficients
+// come from fit_exp2_poly.py (Lawson minimax fit, max relative error 1.0e-4, below the
+// 2^-9 rounding of the bf16 P it feeds); j is added to the exponent field of q(f).  At
+// y = -127 the result packs to exactly +0.
+__device__ __forceinline__ float2 exp2_poly2(float2 y)
+{
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c1 = 0.69328296f, c2 = 0.24221097f, c3 = 0.055008568f;
+    y.x = fmaxf(y.x, -127.0f);
+    y.y = fmaxf(y.y, -127.0f);
+    const float2 t = __fadd2_rn(y, make_float2(kRound, kRound));
+    const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
+    const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), y);
+    float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+    q = __ffma2_rn(q, f, make_float2(c1, c1));
+    q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 // Two floats -> packed bf16x2 (round to nearest even); `lo` lands in bits 0-15.

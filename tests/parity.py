@@ -1,4 +1,7 @@
 """Shared helpers for the GPU parity tests: tolerances and comparisons against the oracle."""
+import json
+import os
+
 import torch
 
 # Tolerances on O and LSE against the fp64 oracle, as stated for this library's target:
@@ -28,6 +31,10 @@ def compare(o_gpu: torch.Tensor, lse_gpu: torch.Tensor, o_ref: torch.Tensor, lse
         # floor set by rounding the exact result to bf16 (shows pure-rounding failures)
         "bf16_floor": (o_ref.to(torch.bfloat16).double() - o_ref).abs().max().item() if o_ref.numel() else 0.0,
     }
+    log = os.environ.get("FA_PARITY_LOG")
+    if log:  # optional record of the margins, one JSON object per comparison
+        with open(log, "a") as f:
+            f.write(json.dumps({"case": what, "test": os.environ.get("PYTEST_CURRENT_TEST", ""), **res}) + "\n")
     assert res["o_max_abs"] <= O_MAX_ABS, f"{what}: {res}"
     assert res["o_mean_abs"] <= O_MEAN_ABS, f"{what}: {res}"
     assert res["lse_max_abs"] <= LSE_MAX_ABS, f"{what}: {res}"

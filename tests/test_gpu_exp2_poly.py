@@ -1,0 +1,64 @@
+"""The FMA-pipe exp2 used for a quarter of the softmax exponentials, checked against 2^x
+in float64 and against the hardware ex2 on the same inputs.
+
+The polynomial's stated bound (fit_exp2_poly.py: max relative error 1.0e-4 on the reduced
+argument) must hold over the whole range the softmax feeds it: x in [-127, 8], plus -inf
+for masked scores, which must give exactly +0.
+"""
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_81_b200 import build as fa_build
+
+pytestmark = pytest.mark.gpu
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+@pytest.fixture(scope="module")
+def probe():
+    td = tempfile.mkdtemp()
+    so = os.path.join(td, "exp2_probe.so")
+    subprocess.check_call([fa_build.nvcc_path(), *fa_build.ARCH_FLAGS, "-O3", "-shared",
+                           "-Xcompiler", "-fPIC", "-I", fa_build.CSRC, "-o", so,
+                           os.path.join(HERE, "csrc", "exp2_probe.cu")])
+    lib = ctypes.CDLL(so)
+    lib.exp2_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int]
+    return lib
+
+
+def run(lib, xs):
+    x = torch.tensor(xs, dtype=torch.float32, device="cuda")
+    poly = torch.empty_like(x)
+    mufu = torch.empty_like(x)
+    assert lib.exp2_probe(x.data_ptr(), poly.data_ptr(), mufu.data_ptr(), x.numel()) == 0
+    return poly.cpu().numpy().astype(np.float64), mufu.cpu().numpy().astype(np.float64)
+
+
+def test_relative_error_over_softmax_range(probe):
+    xs = np.linspace(-126.0, 8.0, 1 << 20, dtype=np.float32)
+    poly, mufu = run(probe, xs)
+    exact = np.exp2(xs.astype(np.float64))
+    rel = np.abs(poly / exact - 1.0)
+    assert rel.max() <= 1.1e-4, rel.max()
+    # no worse than 1.1e-4 relative to the hardware unit either
+    assert np.abs(poly / mufu - 1.0).max() <= 1.2e-4
+
+
+def test_masked_and_underflow(probe):
+    xs = np.array([-np.inf, -np.inf, -127.0, -1000.0, -126.75, -130.0], dtype=np.float32)
+    poly, _ = run(probe, xs)
+    assert poly[0] == 0.0 and poly[1] == 0.0 and poly[2] == 0.0 and poly[3] == 0.0
+    assert (poly[4:] >= 0).all() and (poly[4:] < 2.0 ** -125).all()
+
+
+def test_integers_exact(probe):
+    xs = np.arange(-126, 9, dtype=np.float32)
+    xs = np.concatenate([xs, xs[:1]])[: (len(xs) + 1) // 2 * 2]
+    poly, _ = run(probe, xs)
+    assert np.array_equal(poly, np.exp2(xs.astype(np.float64)))
