@@ -11,7 +11,8 @@
 // staged key/value tile (youngju.dev section 2; toolsku.com generation 2).
 //
 // B200 mapping (one persistent CTA per SM, 12 warps = 3 warpgroups):
-//   warp 8      TMA producer: Q tiles once per work unit, K_j / V_j into an NSTAGE ring
+//   warp 8      TMA producer: Q tiles once per work unit into one of two Q buffers (the
+//               next unit's Q loads while this one runs), K_j / V_j into an NSTAGE ring
 //               of 128-byte-swizzled tiles, completion counted on mbarriers (the warp
 //               runs the loop, one elected lane issues).
 //   warp 9      MMA issuer (warp runs the loop, one elected lane issues):
@@ -29,8 +30,8 @@
 //               softmax warpgroups through setmaxnreg).
 // The two Q tiles of a work unit share their key/value head: two query heads of one
 // group (R even) or two consecutive row tiles of one head (otherwise).  Their MMAs are
-// interleaved S0_j, PV1_{j-1}, S1_j, PV0_j so that the tensor core works on one tile
-// while the softmax warps work on the other.
+// interleaved S0_j, PV1_{j-1}, S1_j, PV0_j -- continued across units -- so that the
+// tensor core works on one tile while the softmax warps work on the other.
 #pragma once
 
 #include <cstdint>
@@ -46,6 +47,7 @@ struct PrefillParams {
     CUtensorMap tm_q;  // (d, Nq, B*Hq) bf16, box (64, 128, 1), 128B swizzle
     CUtensorMap tm_k;  // (d, Nk, B*Hkv)
     CUtensorMap tm_v;  // (d, Nk, B*Hkv)
+    CUtensorMap tm_o;  // (d, Nq, B*Hq) bf16 output, box (64, 128, 1), 128B swizzle
     void *o;
     float *lse;
     int B, Hq, Hkv, Nq, Nk;
@@ -78,13 +80,15 @@ constexpr float kLn2 = 0.6931471805599453f;
 template <int D>
 struct Cfg {
     static constexpr int kTileBytes = 128 * D * 2;
-    static constexpr int kStages = (D == 128) ? 4 : 8;
+    // Q is double-buffered (two sets of the unit's two Q tiles) so the next unit's Q is
+    // loaded while the current one runs; the K/V ring gets what is left of 227 KB.
+    static constexpr int kStages = (D == 128) ? 3 : 8;
     static constexpr int kQOff = 0;
-    static constexpr int kKVOff = 2 * kTileBytes;
+    static constexpr int kKVOff = 4 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-    // barriers: kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], p_ready[2],
-    //           o_done[2], o_free[2], teardown
-    static constexpr int kNumBars = 2 * kStages + 13;
+    // barriers: kv_full[S], kv_empty[S], q_full[2 sets][2], q_empty[2 sets][2], s_full[2],
+    //           p_ready[2], o_done[2], o_free[2], teardown
+    static constexpr int kNumBars = 2 * kStages + 17;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 };
@@ -139,20 +143,34 @@ __device__ __forceinline__ bool decode_unit(const PrefillParams &p, int slot, in
     return true;
 }
 
+// The units of this CTA in order: slots blockIdx.x, blockIdx.x + gridDim.x, ... and, inside
+// a slot, its units k = 0, 1.  Unit index u = 2 * slot + k.
+__device__ __forceinline__ int unit_step(int u) { return u + ((u & 1) ? 2 * (int)gridDim.x - 1 : 1); }
+
+// First valid unit index >= u of this CTA (decoded into w), or -1.
+__device__ __forceinline__ int next_unit(const PrefillParams &p, int u, Unit &w)
+{
+    for (; u < 2 * p.n_slots; u = unit_step(u))
+        if ((u & 1) < units_in_slot(p) && decode_unit(p, u >> 1, u & 1, w)) return u;
+    return -1;
+}
+
 // S = Q K^T over the full head dimension: D/16 MMAs of K = 16.  Both operands are
 // K-major 128-byte-swizzled tiles: 8-row groups 1024 bytes apart (stride offset), a
 // K step of 16 elements advances the start address by 32 bytes inside the swizzle
-// atom, and the second 64-column slab (D = 128) starts 16 KB further on.
+// atom, and the second 64-column slab (D = 128) starts 16 KB further on.  The start
+// address is the descriptor's low field (address >> 4, 14 bits); shared-memory addresses
+// stay below 256 KB, so adding (offset >> 4) to the base descriptor advances it exactly.
 template <int D>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_saddr, uint32_t k_saddr)
 {
     constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, BN, 0);
+    const uint64_t a0 = ptx::smem_desc_sw128(q_saddr, 16, 1024);
+    const uint64_t b0 = ptx::smem_desc_sw128(k_saddr, 16, 1024);
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
-        const uint32_t off = (k >> 2) * kChunkBytes + (k & 3) * 32;
-        const uint64_t a = ptx::smem_desc_sw128(q_saddr + off, 16, 1024);
-        const uint64_t b = ptx::smem_desc_sw128(k_saddr + off, 16, 1024);
-        ptx::mma_ss(d_tmem, a, b, idesc, k > 0 ? 1u : 0u);
+        const uint64_t off = (uint64_t)(((k >> 2) * kChunkBytes + (k & 3) * 32) >> 4);
+        ptx::mma_ss(d_tmem, a0 + off, b0 + off, idesc, k > 0 ? 1u : 0u);
     }
 }
 
@@ -165,18 +183,18 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
                                          bool accumulate)
 {
     constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, D, 1);
+    const uint64_t b0 = ptx::smem_desc_sw128(v_saddr, kChunkBytes, 1024);
 #pragma unroll
-    for (int k = 0; k < BN / 16; ++k) {
-        const uint64_t b = ptx::smem_desc_sw128(v_saddr + k * 2048, kChunkBytes, 1024);
-        ptx::mma_ts(d_tmem, p_tmem + k * 8, b, idesc, (accumulate || k > 0) ? 1u : 0u);
-    }
+    for (int k = 0; k < BN / 16; ++k)
+        ptx::mma_ts(d_tmem, p_tmem + k * 8, b0 + (uint64_t)(k * 2048 >> 4), idesc, (accumulate || k > 0) ? 1u : 0u);
 }
 
 // Pairs of exponentials evaluated on the FMA pipe (exp2_poly2) instead of the MUFU unit:
-// pair c does when kPolyPeriod > 0 and c % kPolyPeriod == kPolyPeriod - 1.  Measured on
-// B200 with this kernel, moving 1/4, 3/8 or 1/2 of them to the FMA pipe made it slower
-// (the softmax is not MUFU-throughput bound here), so the offload is off.
-constexpr int kPolyPeriod = 0;
+// every kPolyPeriod-th pair (0 = none).  The MUFU unit (about 4 exp2 per clock per SM
+// sub-partition) bounds the softmax; measured on B200 with this kernel, one pair in three
+// on the FMA pipe is fastest (one in two runs out of registers, one in four or eight
+// leaves the MUFU the bottleneck).
+constexpr int kPolyPeriod = 3;
 
 // p = 2^(x * sl2 - m) for NC scores of a row held as raw fp32 bits in x[IN .. IN+NC); the
 // p are packed as bf16 pairs into x[OUT .. OUT+NC/2) (OUT <= IN, so every score is read
@@ -195,7 +213,7 @@ __device__ __forceinline__ float exp2_pack(uint32_t (&x)[128], float sl2, float 
     for (int c = 0; c < NC / 2; ++c) {
         const float2 y = __ffma2_rn(make_float2(__uint_as_float(x[IN + 2 * c]), __uint_as_float(x[IN + 2 * c + 1])), c2, nm2);
         float2 e;
-        if (kPolyPeriod > 0 && c % kPolyPeriod == kPolyPeriod - 1) {
+        if (kPolyPeriod > 0 && (c + 1) % (kPolyPeriod > 0 ? kPolyPeriod : 1) == 0) {
             e = ptx::exp2_poly2(y);
         } else {
             e.x = ptx::ex2(y.x);
@@ -266,13 +284,13 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *kv_full = bars;
     uint64_t *kv_empty = bars + C::kStages;
-    uint64_t *q_full = bars + 2 * C::kStages;
-    uint64_t *q_empty = q_full + 2;
-    uint64_t *s_full = q_full + 4;
-    uint64_t *p_ready = q_full + 6;
-    uint64_t *o_done = q_full + 8;
-    uint64_t *o_free = q_full + 10;
-    uint64_t *teardown = q_full + 12;
+    uint64_t *q_full = bars + 2 * C::kStages;  // [set * 2 + tile]
+    uint64_t *q_empty = q_full + 4;             // [set * 2 + tile]
+    uint64_t *s_full = q_full + 8;
+    uint64_t *p_ready = q_full + 10;
+    uint64_t *o_done = q_full + 12;
+    uint64_t *o_free = q_full + 14;
+    uint64_t *teardown = q_full + 16;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
     int *stop_flag = reinterpret_cast<int *>(smem + C::kMiscOff + 4);
 
@@ -286,7 +304,11 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&q_full[s], 1);
-            ptx::mbar_init(&q_empty[s], 1);
+            ptx::mbar_init(&q_full[2 + s], 1);
+            // a Q slot is free again once its last S MMA is done (MMA commit) and the
+            // epilogue, which stages O through the same slot, has stored it (one arrive)
+            ptx::mbar_init(&q_empty[s], 2);
+            ptx::mbar_init(&q_empty[2 + s], 2);
             ptx::mbar_init(&s_full[s], 1);
             ptx::mbar_init(&p_ready[s], 128);
             ptx::mbar_init(&o_done[s], 1);
@@ -320,29 +342,40 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         // issues the copies.
         ptx::regs_decrease<kRegsLow>();
         const bool leader = ptx::elect_one();
-        uint32_t kv_it = 0, q_it = 0;
-        uint32_t q_fills[2] = {0u, 0u};
+        uint32_t kv_it = 0;
+        uint32_t q_fills[4] = {0u, 0u, 0u, 0u};
         bool ok = true;
-        for (int u = blockIdx.x * 2; ok && u < p.n_slots * 2; u += (u & 1) ? 2 * gridDim.x - 1 : 1) {
-            Unit w;
-            if ((u & 1) >= units_in_slot(p) || !decode_unit(p, u >> 1, u & 1, w)) continue;
-            for (int s = 0; s < 2 && ok; ++s) {
-                if (!wait_warp(&q_empty[s], (q_it & 1u) ^ 1u, sf)) { ok = false; break; }
-                ++q_fills[s];
-                if (leader) {
-                    ptx::mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
-                    const int h = s ? w.h1 : w.h0;
-                    const int r = s ? w.r1 : w.r0;
-                    uint8_t *dst = smem + C::kQOff + s * C::kTileBytes;
+        // Q tiles of unit number i (in this CTA's order) go to Q set i & 1 and are loaded one
+        // unit ahead.  The slot of unit i + 1 is released only by unit i - 1's epilogue, so
+        // those loads are issued whenever the slot is free, between K/V loads, without ever
+        // holding up the K/V stream; only at the end of a unit does the warp block on them.
+        auto issue_q = [&](const Unit &uw, uint32_t i, int s) {
+            const int qi = 2 * (int)(i & 1u) + s;
+            ++q_fills[qi];
+            if (leader) {
+                ptx::mbar_arrive_expect_tx(&q_full[qi], C::kTileBytes);
+                const int h = s ? uw.h1 : uw.h0;
+                const int r = s ? uw.r1 : uw.r0;
+                uint8_t *dst = smem + C::kQOff + qi * C::kTileBytes;
 #pragma unroll
-                    for (int c = 0; c < D / 64; ++c)
-                        ptx::tma_load_3d(dst + c * kChunkBytes, &p.tm_q, &q_full[s], 64 * c, r,
-                                         w.b * p.Hq + h);
-                }
-                __syncwarp();
+                for (int c = 0; c < D / 64; ++c)
+                    ptx::tma_load_3d(dst + c * kChunkBytes, &p.tm_q, &q_full[qi], 64 * c, r,
+                                     uw.b * p.Hq + h);
             }
-            if (!ok) break;
-            ++q_it;
+            __syncwarp();
+        };
+        auto q_slot = [&](uint32_t i, int s) { return &q_empty[2 * (int)(i & 1u) + s]; };
+        auto q_free_parity = [&](uint32_t i) { return ((i >> 1) & 1u) ^ 1u; };
+        Unit w, wn;
+        int u = next_unit(p, 2 * (int)blockIdx.x, w);
+        uint32_t i = 0;
+        for (int s = 0; ok && u >= 0 && s < 2; ++s) {
+            if (!wait_warp(q_slot(0, s), q_free_parity(0), sf)) ok = false;
+            else issue_q(w, 0, s);
+        }
+        for (; ok && u >= 0; ++i) {
+            const int un = next_unit(p, unit_step(u), wn);
+            int q_next = (un >= 0) ? 0 : 2;  // look-ahead Q tiles already issued
             const int plane = w.b * p.Hkv + w.g;
             for (int j = 0; j < w.n1 && ok; ++j) {
                 for (int kv = 0; kv < 2; ++kv) {
@@ -360,8 +393,19 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     }
                     __syncwarp();
                     ++kv_it;
+                    while (q_next < 2 &&
+                           __all_sync(0xffffffffu, ptx::mbar_test(q_slot(i + 1, q_next), q_free_parity(i + 1)))) {
+                        issue_q(wn, i + 1, q_next);
+                        ++q_next;
+                    }
                 }
             }
+            for (; ok && q_next < 2; ++q_next) {
+                if (!wait_warp(q_slot(i + 1, q_next), q_free_parity(i + 1), sf)) ok = false;
+                else issue_q(wn, i + 1, q_next);
+            }
+            u = un;
+            w = wn;
         }
         // Let every copy this warp started land before the CTA can exit.
         if (leader) {
@@ -369,8 +413,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 const uint32_t last = kv_it - 1 - ((kv_it - 1 - st) % C::kStages);
                 drain_wait(&kv_full[st], (last / C::kStages) & 1u, p.wait_limit_ns);
             }
-            for (int s = 0; s < 2; ++s)
-                if (q_fills[s] > 0) drain_wait(&q_full[s], (q_fills[s] - 1) & 1u, p.wait_limit_ns);
+            for (int qi = 0; qi < 4; ++qi)
+                if (q_fills[qi] > 0) drain_wait(&q_full[qi], (q_fills[qi] - 1) & 1u, p.wait_limit_ns);
         }
         __syncwarp();
     } else if (warp == 9) {
@@ -383,12 +427,34 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         uint32_t kv_it = 0, units = 0;
         uint32_t p_ph[2] = {0u, 0u};
         bool ok = true;
-        for (int u = blockIdx.x * 2; ok && u < p.n_slots * 2; u += (u & 1) ? 2 * gridDim.x - 1 : 1) {
-            Unit w;
-            if ((u & 1) >= units_in_slot(p) || !decode_unit(p, u >> 1, u & 1, w)) continue;
-            const uint32_t q_par = units & 1u;
-            const uint32_t free_par = q_par ^ 1u;  // first unit passes at once
-            if (!wait_warp(&q_full[0], q_par, sf) || !wait_warp(&q_full[1], q_par, sf)) break;
+        // The P V of tile 1's last key tile is not issued at the end of its unit but carried
+        // into the next unit's first iteration, after that unit's first S0 MMA: the
+        // S0 / PV1 / S1 / PV0 ping-pong then runs on across unit boundaries instead of
+        // draining the tensor pipe at every unit.
+        bool pend = false, pend_acc = false, pend_free = false;
+        uint32_t pend_v = 0, pend_free_par = 0;
+        auto issue_pv1 = [&](uint32_t v_stage, bool acc, bool need_free, uint32_t fpar, bool last) -> bool {
+            if (!wait_warp(&p_ready[1], p_ph[1], sf)) return false;
+            p_ph[1] ^= 1u;
+            if (need_free && !wait_warp(&o_free[1], fpar, sf)) return false;
+            ptx::tc_fence_after();
+            if (leader) {
+                issue_pv<D>(tmem + 384, tmem + 128, kv_saddr0 + v_stage * C::kTileBytes, acc);
+                ptx::mma_commit(&kv_empty[v_stage]);
+                if (last) ptx::mma_commit(&o_done[1]);
+            }
+            __syncwarp();
+            return true;
+        };
+        Unit w;
+        for (int u = next_unit(p, 2 * (int)blockIdx.x, w); ok && u >= 0; u = next_unit(p, unit_step(u), w)) {
+            const uint32_t free_par = (units & 1u) ^ 1u;  // first unit passes at once
+            const uint32_t qset = units & 1u;
+            const uint32_t q_par = (units >> 1) & 1u;
+            uint64_t *qf = q_full + 2 * qset;
+            uint64_t *qe = q_empty + 2 * qset;
+            const uint32_t q_saddr = q_saddr0 + 2 * qset * C::kTileBytes;
+            if (!wait_warp(&qf[0], q_par, sf) || !wait_warp(&qf[1], q_par, sf)) break;
             ptx::tc_fence_after();
             uint32_t prev_v = 0;
             for (int j = 0; j < w.n1; ++j) {
@@ -401,28 +467,23 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 const uint32_t k_saddr = kv_saddr0 + ks * C::kTileBytes;
                 if (j < w.n0) {
                     if (leader) {
-                        issue_qk<D>(tmem + 0, q_saddr0, k_saddr);
+                        issue_qk<D>(tmem + 0, q_saddr, k_saddr);
                         if (signal_s) ptx::mma_commit(&s_full[0]);
-                        if (j == w.n0 - 1) ptx::mma_commit(&q_empty[0]);
+                        if (j == w.n0 - 1) ptx::mma_commit(&qe[0]);
                     }
                     __syncwarp();
                 }
                 if (j > 0) {
-                    if (!wait_warp(&p_ready[1], p_ph[1], sf)) { ok = false; break; }
-                    p_ph[1] ^= 1u;
-                    if (j - 1 == 0 && !wait_warp(&o_free[1], free_par, sf)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    if (leader) {
-                        issue_pv<D>(tmem + 384, tmem + 128, kv_saddr0 + prev_v * C::kTileBytes, j - 1 > 0);
-                        ptx::mma_commit(&kv_empty[prev_v]);
-                    }
-                    __syncwarp();
+                    if (!issue_pv1(prev_v, j - 1 > 0, j - 1 == 0, free_par, false)) { ok = false; break; }
+                } else if (pend) {
+                    if (!issue_pv1(pend_v, pend_acc, pend_free, pend_free_par, true)) { ok = false; break; }
+                    pend = false;
                 }
                 if (leader) {
-                    issue_qk<D>(tmem + 128, q_saddr0 + C::kTileBytes, k_saddr);
+                    issue_qk<D>(tmem + 128, q_saddr + C::kTileBytes, k_saddr);
                     if (signal_s) ptx::mma_commit(&s_full[1]);
                     ptx::mma_commit(&kv_empty[ks]);
-                    if (j == w.n1 - 1) ptx::mma_commit(&q_empty[1]);
+                    if (j == w.n1 - 1) ptx::mma_commit(&qe[1]);
                 }
                 __syncwarp();
                 if (!wait_warp(&kv_full[vs], vph, sf)) { ok = false; break; }
@@ -441,19 +502,14 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 kv_it += 2;
             }
             if (!ok) break;
-            // last P V of tile 1
-            if (!wait_warp(&p_ready[1], p_ph[1], sf)) break;
-            p_ph[1] ^= 1u;
-            if (w.n1 == 1 && !wait_warp(&o_free[1], free_par, sf)) break;
-            ptx::tc_fence_after();
-            if (leader) {
-                issue_pv<D>(tmem + 384, tmem + 128, kv_saddr0 + prev_v * C::kTileBytes, w.n1 > 1);
-                ptx::mma_commit(&kv_empty[prev_v]);
-                ptx::mma_commit(&o_done[1]);
-            }
-            __syncwarp();
+            pend = true;
+            pend_v = prev_v;
+            pend_acc = w.n1 > 1;
+            pend_free = w.n1 == 1;
+            pend_free_par = free_par;
             ++units;
         }
+        if (ok && pend) issue_pv1(pend_v, pend_acc, pend_free, pend_free_par, true);
         // Every MMA and commit issued above completes before the CTA can exit.
         if (leader) {
             ptx::mma_commit(teardown);
@@ -470,9 +526,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         const uint32_t tO = tmem + lane_base + 256u + 128u * s;  // O_s
         const float sl2 = p.scale_log2;
         uint32_t s_ph = 0, units = 0;
-        for (int u = blockIdx.x * 2; u < p.n_slots * 2; u += (u & 1) ? 2 * gridDim.x - 1 : 1) {
-            Unit w;
-            if ((u & 1) >= units_in_slot(p) || !decode_unit(p, u >> 1, u & 1, w)) continue;
+        Unit w;
+        for (int u = next_unit(p, 2 * (int)blockIdx.x, w); u >= 0; u = next_unit(p, unit_step(u), w)) {
             const int h = s ? w.h1 : w.h0;
             const int r0 = s ? w.r1 : w.r0;
             const int n = s ? w.n1 : w.n0;
@@ -536,17 +591,24 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             }
             if (!ok) break;
             // ------------------------------------------------------------- epilogue
+            // O_s / lo leaves TMEM as soon as it is read (o_free lets the next unit's first
+            // P V overwrite it).  bf16 output is staged, 128-byte swizzled, in this unit's Q
+            // slot -- no MMA reads it any more -- and written by one TMA store; the slot is
+            // then handed back to the producer.  fp32 output is stored row by row.
             if (!wait_warp(&o_done[s], units & 1u, sf)) break;
             ptx::tc_fence_after();
             const bool valid = row < p.Nq;
             const float inv_l = 1.f / lo;
             const size_t orow = ((size_t)w.b * p.Hq + h) * (size_t)p.Nq + (size_t)(valid ? row : 0);
+            const int qi = 2 * (int)(units & 1u) + s;
             uint32_t ov[D];
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(tO + 32 * c, &ov[32 * c]);
             ptx::tmem_wait_ld();
-            if (valid) {
-                if (OUT_F32) {
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&o_free[s]);
+            if (OUT_F32) {
+                if (valid) {
                     float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D);
 #pragma unroll
                     for (int e = 0; e < D / 4; ++e)
@@ -554,24 +616,37 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                                              __uint_as_float(ov[4 * e + 1]) * inv_l,
                                              __uint_as_float(ov[4 * e + 2]) * inv_l,
                                              __uint_as_float(ov[4 * e + 3]) * inv_l);
-                } else {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D);
+                }
+                if (tid == 0) ptx::mbar_arrive(&q_empty[qi]);
+            } else {
+                uint8_t *stage = smem + C::kQOff + qi * C::kTileBytes;
 #pragma unroll
-                    for (int e = 0; e < D / 8; ++e) {
-                        uint4 v4;
-                        v4.x = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
-                        v4.y = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
-                        v4.z = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
-                        v4.w = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
-                        dst[e] = v4;
-                    }
+                for (int e = 0; e < D / 8; ++e) {
+                    uint4 v4;
+                    v4.x = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
+                    v4.y = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
+                    v4.z = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
+                    v4.w = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
+                    // 16-byte chunk e of the row: slab e / 8, chunk (e % 8) swizzled by row % 8
+                    const int slab = e >> 3, chunk = (e & 7) ^ (tid & 7);
+                    *reinterpret_cast<uint4 *>(stage + slab * kChunkBytes + tid * 128 + chunk * 16) = v4;
+                }
+                ptx::fence_proxy_async_smem();
+                if (s == 0) ptx::named_barrier_sync<1, 128>();
+                else ptx::named_barrier_sync<2, 128>();
+                if (tid == 0) {
+#pragma unroll
+                    for (int c = 0; c < D / 64; ++c)
+                        ptx::tma_store_3d(&p.tm_o, stage + c * kChunkBytes, 64 * c, r0, w.b * p.Hq + h);
+                    ptx::bulk_commit_group();
+                    ptx::bulk_wait_group_read0();
+                    ptx::mbar_arrive(&q_empty[qi]);
                 }
             }
             if (valid) p.lse[orow] = (m + ptx::lg2(l)) * kLn2;
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&o_free[s]);
             ++units;
         }
+        if (!OUT_F32 && tid == 0) ptx::bulk_wait_group0();  // stores complete before exit
     }
 
     else {
