@@ -49,6 +49,7 @@ struct DeviceInfo {
     bool sm100 = false;
     int num_sms = 0;
     bool prefill_attr_set[2][2] = {{false, false}, {false, false}};
+    bool decode_attr_set[2][4] = {{false, false, false, false}, {false, false, false, false}};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -98,14 +99,16 @@ EncodeTiledFn get_encode_fn()
     return fn;
 }
 
-// A (D, rows, planes) bf16 tensor with 128-row boxes of 64 columns, 128-byte swizzle.
-int encode_rows_map(CUtensorMap *m, const void *base, int D, long long rows, long long planes)
+// A (D, rows, planes) bf16 tensor with boxes of `box_rows` rows x 64 columns, 128-byte
+// swizzle.
+int encode_rows_map(CUtensorMap *m, const void *base, int D, long long rows, long long planes,
+                    unsigned box_rows = 128)
 {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -222,21 +225,39 @@ size_t decode_ws_bytes(int B, int Hq, int Nmax, int d)
     return align256((size_t)B * Hq * S * d * sizeof(float)) + align256((size_t)B * Hq * S * sizeof(float));
 }
 
+// Persistent split kernel: one CTA per SM (at most one per work item).
 template <int D, int RG>
-void launch_split(const fa::DecodeParams &p, cudaStream_t st)
+int launch_split(fa::DecodeParams p, DeviceInfo *info, cudaStream_t st)
 {
-    dim3 grid(p.S_max, p.Hq / RG, p.B);
-    fa::fa_decode_split_kernel<D, RG><<<grid, fa::decode::kThreads, 0, st>>>(p);
+    using C = fa::decode::SplitCfg<D, RG>;
+    static_assert(C::kSmemBytes * fa::decode::kCtasPerSm <= 227 * 1024, "decode CTAs per SM do not fit");
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        bool &set = info->decode_attr_set[D == 128][RG == 8 ? 3 : RG == 4 ? 2 : RG == 2 ? 1 : 0];
+        if (!set) {
+            cudaError_t e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, RG>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+            if (e != cudaSuccess)
+                return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+            set = true;
+        }
+    }
+    p.n_hg = p.Hq / RG;
+    p.n_items = p.S_max * p.B * p.n_hg;
+    const int max_ctas = fa::decode::kCtasPerSm * info->num_sms;
+    const int grid = p.n_items < max_ctas ? p.n_items : max_ctas;
+    fa::fa_decode_split_kernel<D, RG><<<grid, fa::decode::kThreads, C::kSmemBytes, st>>>(p);
+    return FA_OK;
 }
 
 template <int D>
-void launch_split_rg(const fa::DecodeParams &p, int rg, cudaStream_t st)
+int launch_split_rg(const fa::DecodeParams &p, int rg, DeviceInfo *info, cudaStream_t st)
 {
     switch (rg) {
-    case 8: launch_split<D, 8>(p, st); break;
-    case 4: launch_split<D, 4>(p, st); break;
-    case 2: launch_split<D, 2>(p, st); break;
-    default: launch_split<D, 1>(p, st); break;
+    case 8: return launch_split<D, 8>(p, info, st);
+    case 4: return launch_split<D, 4>(p, info, st);
+    case 2: return launch_split<D, 2>(p, info, st);
+    default: return launch_split<D, 1>(p, info, st);
     }
 }
 
@@ -312,8 +333,8 @@ int fa_decode(const void *q, const void *kcache, const void *vcache, const int *
     fa::DecodeParams p;
     memset(&p, 0, sizeof p);
     p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.kc = static_cast<const __nv_bfloat16 *>(kcache);
-    p.vc = static_cast<const __nv_bfloat16 *>(vcache);
+    if ((rc = encode_rows_map(&p.tm_k, kcache, d, Nmax, (long long)B * Hkv, fa::decode::kSub)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, vcache, d, Nmax, (long long)B * Hkv, fa::decode::kSub)) != FA_OK) return rc;
     p.seqlens = seqlens;
     p.S_max = (int)decode_splits(Nmax);
     p.part_o = static_cast<float *>(workspace);
@@ -329,8 +350,9 @@ int fa_decode(const void *q, const void *kcache, const void *vcache, const int *
     p.scale_log2 = scale * 1.4426950408889634f;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (d == 128) launch_split_rg<128>(p, rg, st);
-    else launch_split_rg<64>(p, rg, st);
+    p.wait_limit_ns = g_wait_limit_ns;
+    rc = (d == 128) ? launch_split_rg<128>(p, rg, info, st) : launch_split_rg<64>(p, rg, info, st);
+    if (rc != FA_OK) return rc;
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
     e = (d == 128) ? launch_merge<128>(p, st) : launch_merge<64>(p, st);
@@ -402,8 +424,8 @@ int fa_decode_noalloc(const void *q, const void *kcache, const void *vcache, con
     fa::DecodeParams p;
     memset(&p, 0, sizeof p);
     p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.kc = static_cast<const __nv_bfloat16 *>(kcache);
-    p.vc = static_cast<const __nv_bfloat16 *>(vcache);
+    if ((rc = encode_rows_map(&p.tm_k, kcache, d, Nmax, (long long)B * Hkv, fa::decode::kSub)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, vcache, d, Nmax, (long long)B * Hkv, fa::decode::kSub)) != FA_OK) return rc;
     p.seqlens = seqlens;
     p.S_max = (int)decode_splits(Nmax);
     p.part_o = static_cast<float *>(scratch);
@@ -419,8 +441,9 @@ int fa_decode_noalloc(const void *q, const void *kcache, const void *vcache, con
     p.scale_log2 = scale * 1.4426950408889634f;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (d == 128) launch_split_rg<128>(p, rg, st);
-    else launch_split_rg<64>(p, rg, st);
+    p.wait_limit_ns = g_wait_limit_ns;
+    rc = (d == 128) ? launch_split_rg<128>(p, rg, info, st) : launch_split_rg<64>(p, rg, info, st);
+    if (rc != FA_OK) return rc;
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
     e = (d == 128) ? launch_merge<128>(p, st) : launch_merge<64>(p, st);

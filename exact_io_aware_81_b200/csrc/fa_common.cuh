@@ -72,4 +72,22 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const 
     }
 }
 
+// A barrier among the warps of a role built on an mbarrier (initialised with a count of
+// one arrival per warp), so that -- unlike bar.sync -- waiting on it is time-bounded and
+// honours the CTA stop flag.  Every participating warp calls sync() the same number of
+// times; each call is one phase.
+struct GroupBarrier {
+    uint64_t *bar;
+    uint32_t phase;
+
+    __device__ __forceinline__ bool sync(const StopFlag &sf)
+    {
+        __syncwarp();
+        if ((threadIdx.x & 31u) == 0u) ptx::mbar_arrive(bar);
+        const bool ok = wait_warp(bar, phase, sf);
+        phase ^= 1u;
+        return ok;
+    }
+};
+
 }  // namespace fa

@@ -3,15 +3,17 @@
 // Decode (one new query row per sequence) reads the whole cache every step and does
 // only 4 flops per byte, so it is bound by HBM bandwidth (youngju.dev "attention
 // variants", section 7).  The cache of one (sequence, key/value head) is contiguous, so
-// it is cut into chunks of kChunk keys that independent CTAs stream in parallel:
+// it is cut into chunks of kChunk keys, each an independent work item:
 //
-//   split kernel, one CTA per (chunk, group of RG query heads of one KV head, sequence):
-//     K pass: each lane reads one 16-byte slice of a key row (fully coalesced, several
-//             loads in flight), scores for the RG heads are reduced across the lanes of
-//             the row; scores (pre-multiplied by scale*log2 e) go to shared memory.
-//     softmax of the chunk: max, p = 2^(s - max), sum.
-//     V pass: the same slicing over value rows, O_part += p * v in fp32.
-//     writes the normalised partial output and its log2-sum-exp to the workspace.
+//   split kernel (persistent, one CTA per SM): a producer warp streams every item's key
+//     rows and then its value rows into a ring of shared-memory stages of kSub rows with
+//     1-D TMA bulk copies (completion counted in bytes on mbarriers), running up to a
+//     ring's worth of bytes ahead; eight consumer warps take the stages in order:
+//     K pass: 16-byte slices of a key row per lane, scores of the item's RG query heads
+//             (scale * log2 e folded into q) reduced across the lanes of the row;
+//     chunk softmax: max, p = 2^(s - max), sum;
+//     V pass: the same slicing over value rows, O_part += p * v in fp32;
+//     then the normalised partial output and its log2-sum-exp go to the workspace.
 //   merge kernel, one CTA per (head, sequence): M = max of the partial log-sum-exps,
 //     w_s = 2^(lse_s - M), o = sum_s w_s o_s / sum_s w_s, lse = M + log2 sum_s w_s.
 // The merge is the same rescaling the online softmax applies between key blocks
@@ -27,264 +29,305 @@
 namespace fa {
 
 struct DecodeParams {
+    CUtensorMap tm_k;         // kcache as (D, Nmax, B*Hkv) bf16, box (64, 64, 1), 128B swizzle
+    CUtensorMap tm_v;         // vcache, same shape
     const __nv_bfloat16 *q;   // (B, Hq, D)
-    const __nv_bfloat16 *kc;  // (B, Hkv, Nmax, D)
-    const __nv_bfloat16 *vc;  // (B, Hkv, Nmax, D)
     const int *seqlens;       // (B)
     float *part_o;            // (B, Hq, S_max, D)  normalised partial outputs
     float *part_lse;          // (B, Hq, S_max)     partial log2-sum-exp (scaled scores)
     __nv_bfloat16 *o;         // (B, Hq, D)
     float *lse;               // (B, Hq) natural log, may be null
     int B, Hq, Hkv, Nmax, R, S_max;
+    int n_hg;      // head groups: Hq / RG
+    int n_items;   // S_max * B * n_hg candidate work items (chunk-major order)
     float scale_log2;
+    unsigned long long wait_limit_ns;
 };
 
 namespace decode {
 
-constexpr int kChunk = 256;
-constexpr int kThreads = 128;
-constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 8;
+constexpr int kChunk = 256;        // keys per work item
+constexpr int kSub = 64;           // key rows per ring stage (one TMA box per 64 columns)
+constexpr int kWarps = 4;          // consumer warps
+constexpr int kThreads = 32 * (kWarps + 1);
+constexpr int kCtasPerSm = 3;
+constexpr int kBoxBytes = kSub * 128;  // 64 rows x 64 bf16 columns
 constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D, int RG>
+struct SplitCfg {
+    static constexpr int kStageBytes = (D / 64) * kBoxBytes;
+    static constexpr int kStages = (D == 128) ? 4 : 8;                 // 64 KB ring
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kScoreOff = kRingBytes;                       // float [RG][kChunk]
+    static constexpr int kMOff = kScoreOff + RG * kChunk * 4;          // float m[RG], l[RG]
+    static constexpr int kBarOff = (kMOff + 2 * RG * 4 + 15) & ~15;    // full[S], empty[S], group
+    static constexpr int kStopOff = kBarOff + (2 * kStages + 1) * 8;
+    static constexpr int kSmemBytes = kStopOff + 16 + 1024;            // + alignment slack
+};
 
 __device__ __forceinline__ int clamp_len(int L, int Nmax)
 {
     return L < 0 ? 0 : (L > Nmax ? Nmax : L);
 }
 
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8])
+// Byte offset of 16-byte chunk `c` (8 bf16 of the row, 0 .. D/8-1) of row `r` of a stage
+// written by TMA with 128-byte swizzle: 64-column boxes of 64 rows x 128 bytes, the
+// chunk index XORed with the row's index modulo 8.
+__device__ __forceinline__ uint32_t stage_offset(int r, int c)
 {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
+    return (uint32_t)((c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-__device__ __forceinline__ void unpack8x2(const uint4 &u, float2 (&f)[4])
-{
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-}
-
-// Sums V values per lane over the LPK lanes that share one key row and scatters the
-// results: after the call lane `sub` holds, in a[0], the full sum of value head_of(sub).
-// Levels with more than one value left halve the values (a lane keeps one half and adds
-// its partner's copy of that half), the remaining levels are plain butterflies.
-template <int V, int LPK>
-__device__ __forceinline__ void reduce_scatter(float (&a)[V], int sub)
-{
-    int n = V;
-#pragma unroll
-    for (int off = LPK / 2; off >= 1; off >>= 1) {
-        if (n > 1) {
-            const int half = n >> 1;
-            const bool upper = (sub & off) != 0;
-#pragma unroll
-            for (int i = 0; i < V / 2; ++i) {
-                if (i < half) {
-                    const float send = upper ? a[i] : a[i + half];
-                    const float keep = upper ? a[i + half] : a[i];
-                    a[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-                }
-            }
-            n = half;
-        } else {
-            a[0] += __shfl_xor_sync(0xffffffffu, a[0], off);
-        }
-    }
-}
-
-// Which value lane `sub` holds after reduce_scatter<V, LPK>, and whether it is the one
-// lane (of the group holding that value) that writes it.
-template <int V, int LPK>
-__device__ __forceinline__ int scatter_head(int sub, bool &writer)
-{
-    int head = 0, n = V, low_mask = 0;
-#pragma unroll
-    for (int off = LPK / 2; off >= 1; off >>= 1) {
-        if (n > 1) {
-            n >>= 1;
-            if (sub & off) head += n;
-        } else {
-            low_mask |= off;
-        }
-    }
-    writer = (sub & low_mask) == 0;
-    return head;
-}
-
-__device__ __forceinline__ uint4 ldg_stream(const void *p)
-{
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) { return ptx::pack_bf16x2(lo, hi); }
 
 }  // namespace decode
 
-// D: head dim (64 or 128).  RG: query heads per CTA (all of one KV head).
+// Work item `it` (chunk-major: the early chunks, valid for every sequence, come first, so
+// a round-robin over the persistent CTAs gives each a similar mix): returns false if the
+// chunk starts past the sequence's length.
+__device__ __forceinline__ bool decode_item(const DecodeParams &p, int it, int &b, int &hg, int &start, int &n)
+{
+    const int bh = p.B * p.n_hg;
+    const int chunk = it / bh;
+    const int rest = it - chunk * bh;
+    b = rest / p.n_hg;
+    hg = rest - b * p.n_hg;
+    const int L = decode::clamp_len(p.seqlens[b], p.Nmax);
+    start = chunk * decode::kChunk;
+    if (start >= L) return false;
+    n = min(decode::kChunk, L - start);
+    return true;
+}
+
+// Split kernel.  D: head dim (64 or 128).  RG: query heads per work item (<= 8, all of one
+// KV head).  The RG query rows are the rows of the M = 16 operand of mma.sync m16n8k16
+// (rows RG .. 15 are zero): S = Q K^T per 8-key column tile, O += P V per 8-column tile,
+// both with fp32 accumulation; K and V fragments come from the swizzled stages through
+// ldmatrix (transposed for V).
 template <int D, int RG>
-__global__ void __launch_bounds__(decode::kThreads)
+__global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
     fa_decode_split_kernel(const __grid_constant__ DecodeParams p)
 {
     using namespace decode;
-    constexpr int LPK = D / 8;      // lanes per key row (16 bytes each)
-    constexpr int KPW = 32 / LPK;   // key rows per warp instruction
-    constexpr int KPI = KPW * kWarps;  // key rows per CTA instruction
+    using C = SplitCfg<D, RG>;
+    static_assert(RG <= 8, "at most 8 query heads per item");
+    constexpr int KSTEPS = D / 16;          // k-steps of S = Q K^T
+    constexpr int NT = D / 8 / kWarps;      // 8-column tiles of O per consumer warp
 
-    __shared__ float s_sm[RG][kChunk];
-    __shared__ float red[kWarps][RG][D];
-    __shared__ float m_sm[RG], l_sm[RG];
-
-    // let the merge kernel (launched as a programmatic dependent) get scheduled early; it
-    // waits for this whole grid to finish before it reads any partial
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int chunk = blockIdx.x;
-    const int h0 = blockIdx.y * RG;
-    const int b = blockIdx.z;
-    const int raw = p.seqlens[b];
-    const int L = clamp_len(raw, p.Nmax);
-    if (raw != L && chunk == 0 && blockIdx.y == 0 && threadIdx.x == 0) raise_error(kErrSeqlenRange);
-    const int start = chunk * kChunk;
-    if (start >= L) return;
-    const int n = min(kChunk, L - start);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    float(*s_sm)[kChunk] = reinterpret_cast<float(*)[kChunk]>(smem + C::kScoreOff);
+    float *m_sm = reinterpret_cast<float *>(smem + C::kMOff);
+    float *l_sm = m_sm + RG;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *empty = full + C::kStages;
+    uint64_t *group = empty + C::kStages;  // consumer-warp barrier
+    int *stop_flag = reinterpret_cast<int *>(smem + C::kStopOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int sub = lane % LPK;   // which 16-byte slice of the row
-    const int kk = lane / LPK;    // which row of the warp's group
-    const int g = h0 / p.R;
-
-    const size_t plane = ((size_t)b * p.Hkv + g) * (size_t)p.Nmax + (size_t)start;
-    const __nv_bfloat16 *kbase = p.kc + plane * D + sub * 8;
-    const __nv_bfloat16 *vbase = p.vc + plane * D + sub * 8;
-
-    float2 qf[RG][4];
-#pragma unroll
-    for (int r = 0; r < RG; ++r) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(p.q + ((size_t)b * p.Hq + h0 + r) * D + sub * 8);
-        unpack8x2(u, qf[r]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) qf[r][e] = __fmul2_rn(qf[r][e], make_float2(p.scale_log2, p.scale_log2));
-    }
-    bool writer;
-    const int my_head = scatter_head<RG, LPK>(sub, writer);
-
-    // ---------------------------------------------------------------- K pass
-    for (int base = 0; base < n; base += KPI * kUnroll) {
-        uint4 kr[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int key = base + u * KPI + warp * KPW + kk;
-            kr[u] = key < n ? ldg_stream(kbase + (size_t)key * D) : make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::kStages; ++i) {
+            ptx::mbar_init(&full[i], 1);
+            ptx::mbar_init(&empty[i], kWarps);
         }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int key = base + u * KPI + warp * KPW + kk;
-            float2 kf[4];
-            unpack8x2(kr[u], kf);
-            float acc[RG];
-#pragma unroll
-            for (int r = 0; r < RG; ++r) {
-                float2 a = __fmul2_rn(qf[r][0], kf[0]);
-#pragma unroll
-                for (int e = 1; e < 4; ++e) a = __ffma2_rn(qf[r][e], kf[e], a);
-                acc[r] = a.x + a.y;
-            }
-            reduce_scatter<RG, LPK>(acc, sub);
-            if (writer && key < n) s_sm[my_head][key] = acc[0];
-        }
+        ptx::mbar_init(group, kWarps);
+        *stop_flag = 0;
+        ptx::fence_barrier_init();
     }
     __syncthreads();
-
-    // ------------------------------------------------------- chunk softmax
-    for (int r = warp; r < RG; r += kWarps) {
-        float mx = -INFINITY;
-        for (int k = lane; k < n; k += 32) mx = fmaxf(mx, s_sm[r][k]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        float sum = 0.f;
-        for (int k = lane; k < n; k += 32) {
-            const float e = ptx::ex2(s_sm[r][k] - mx);
-            s_sm[r][k] = e;
-            sum += e;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane == 0) {
-            m_sm[r] = mx;
-            l_sm[r] = sum;
-        }
+    // let the merge kernel (launched as a programmatic dependent) get scheduled early; it
+    // waits for this whole grid to finish before it reads any partial
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const StopFlag sf{stop_flag, p.wait_limit_ns};
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        for (int b = 0; b < p.B; ++b)
+            if (p.seqlens[b] != clamp_len(p.seqlens[b], p.Nmax)) raise_error(kErrSeqlenRange);
     }
-    __syncthreads();
 
-    // ---------------------------------------------------------------- V pass
-    float2 acc[RG][4];
-#pragma unroll
-    for (int r = 0; r < RG; ++r)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[r][e] = make_float2(0.f, 0.f);
-    for (int base = 0; base < n; base += KPI * kUnroll) {
-        uint4 vr[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int key = base + u * KPI + warp * KPW + kk;
-            vr[u] = key < n ? ldg_stream(vbase + (size_t)key * D) : make_uint4(0, 0, 0, 0);
+    if (warp == kWarps) {
+        // ------------------------------------------------------------- producer
+        const bool leader = ptx::elect_one();
+        if (leader) {
+            ptx::tma_prefetch_desc(&p.tm_k);
+            ptx::tma_prefetch_desc(&p.tm_v);
         }
+        uint32_t ring = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+            int b, hg, start, n;
+            if (!decode_item(p, it, b, hg, start, n)) continue;
+            const int plane = b * p.Hkv + hg * RG / p.R;
+            for (int pass = 0; pass < 2 && ok; ++pass) {
+                const CUtensorMap *map = pass ? &p.tm_v : &p.tm_k;
+                for (int t = 0; t * kSub < n; ++t) {
+                    const uint32_t st = ring % C::kStages;
+                    const uint32_t ph = (ring / C::kStages) & 1u;
+                    if (!wait_warp(&empty[st], ph ^ 1u, sf)) { ok = false; break; }
+                    if (leader) {
+                        ptx::mbar_arrive_expect_tx(&full[st], C::kStageBytes);
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int key = base + u * KPI + warp * KPW + kk;
-            if (key < n) {
-                float2 vf[4];
-                unpack8x2(vr[u], vf);
-#pragma unroll
-                for (int r = 0; r < RG; ++r) {
-                    const float pr = s_sm[r][key];
-                    const float2 p2 = make_float2(pr, pr);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[r][e] = __ffma2_rn(p2, vf[e], acc[r][e]);
+                        for (int c = 0; c < D / 64; ++c)
+                            ptx::tma_load_3d(smem + st * C::kStageBytes + c * kBoxBytes, map, &full[st],
+                                             64 * c, start + t * kSub, plane);
+                    }
+                    __syncwarp();
+                    ++ring;
                 }
             }
         }
-    }
-    // rows handled by different lanes of a warp -> lanes with kk == 0
-#pragma unroll
-    for (int off = LPK; off < 32; off <<= 1)
-#pragma unroll
-        for (int r = 0; r < RG; ++r)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                acc[r][e].x += __shfl_xor_sync(0xffffffffu, acc[r][e].x, off);
-                acc[r][e].y += __shfl_xor_sync(0xffffffffu, acc[r][e].y, off);
+        // let every copy issued above land before the CTA can exit
+        if (leader) {
+            for (uint32_t st = 0; st < (uint32_t)C::kStages && st < ring; ++st) {
+                const uint32_t last = ring - 1 - ((ring - 1 - st) % C::kStages);
+                const uint32_t par = (last / C::kStages) & 1u;
+                const uint64_t t0 = ptx::globaltimer_ns();
+                while (!ptx::mbar_test(&full[st], par))
+                    if (ptx::globaltimer_ns() - t0 > p.wait_limit_ns) { raise_error(kErrTimeout); break; }
             }
-    if (kk == 0) {
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------- consumers
+        const int gid = lane >> 2;   // fragment row (query head) / ldmatrix row group
+        const int tig = lane & 3;    // thread in group
+        const bool row_real = gid < RG;
+        GroupBarrier gb{group, 0u};
+        uint32_t ring = 0;
+        // ldmatrix addressing: lane supplies row (lane & 7) of matrix (lane >> 3)
+        const int lm_row = lane & 7;
+        const int lm_mat = lane >> 3;
+        for (int it = blockIdx.x; it < p.n_items; it += gridDim.x) {
+            int b, hg, start, n;
+            if (!decode_item(p, it, b, hg, start, n)) continue;
+            const int h0 = hg * RG;
+            // A operand of S = Q K^T: row gid = query head h0 + gid (zero beyond RG)
+            uint32_t qa[KSTEPS][2];
+            {
+                const uint32_t *qrow = reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + h0 + (row_real ? gid : 0)) * D);
 #pragma unroll
-        for (int r = 0; r < RG; ++r)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                red[warp][r][sub * 8 + 2 * e] = acc[r][e].x;
-                red[warp][r][sub * 8 + 2 * e + 1] = acc[r][e].y;
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    qa[ks][0] = row_real ? qrow[8 * ks + tig] : 0u;
+                    qa[ks][1] = row_real ? qrow[8 * ks + 4 + tig] : 0u;
+                }
             }
+            bool ok = true;
+            // ------------------------------------------------------------ K pass
+            for (int t = 0; t * kSub < n; ++t) {
+                const uint32_t st = ring % C::kStages;
+                if (!wait_warp(&full[st], (ring / C::kStages) & 1u, sf)) { ok = false; break; }
+                const uint32_t sbase = ptx::smem_addr(smem + st * C::kStageBytes);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int key0 = warp * 16 + nt * 8;  // 8 keys of this column tile
+                    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < KSTEPS; ks += 2) {
+                        uint32_t b0, b1, b2, b3;
+                        ptx::ldsm_x4(sbase + stage_offset(key0 + lm_row, 2 * ks + lm_mat), b0, b1, b2, b3);
+                        const uint32_t a0[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
+                        const uint32_t a1[4] = {qa[ks + 1][0], 0u, qa[ks + 1][1], 0u};
+                        ptx::mma_16816_bf16(c, a0, b0, b1);
+                        ptx::mma_16816_bf16(c, a1, b2, b3);
+                    }
+                    if (row_real) {
+                        const int key = t * kSub + key0 + 2 * tig;
+                        s_sm[gid][key] = key < n ? c[0] * p.scale_log2 : -INFINITY;
+                        s_sm[gid][key + 1] = key + 1 < n ? c[1] * p.scale_log2 : -INFINITY;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&empty[st]);
+                ++ring;
+            }
+            if (!ok || !gb.sync(sf)) break;
+            // ------------------------------------------------------ chunk softmax
+            for (int r = warp; r < RG; r += kWarps) {
+                float mx = -INFINITY;
+                for (int k = lane; k < n; k += 32) mx = fmaxf(mx, s_sm[r][k]);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                float sum = 0.f;
+                for (int k = lane; k < kChunk; k += 32) {
+                    const float e = k < n ? ptx::ex2(s_sm[r][k] - mx) : 0.f;
+                    s_sm[r][k] = e;
+                    sum += e;
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                if (lane == 0) {
+                    m_sm[r] = mx;
+                    l_sm[r] = sum;
+                }
+            }
+            if (!gb.sync(sf)) break;
+            // ------------------------------------------------------------ V pass
+            float acc[NT][4];
+#pragma unroll
+            for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+            for (int t = 0; t * kSub < n; ++t) {
+                const uint32_t st = ring % C::kStages;
+                if (!wait_warp(&full[st], (ring / C::kStages) & 1u, sf)) { ok = false; break; }
+                uint8_t *stage = smem + st * C::kStageBytes;
+                const int rows = min(kSub, n - t * kSub);
+                if (rows < kSub) {
+                    // rows past the sequence hold whatever the cache holds there: clear them
+                    // so that their zero weights cannot meet a non-finite value (and order
+                    // these writes before the copy engine refills the stage)
+                    for (int idx = threadIdx.x; idx < (kSub - rows) * (D / 8); idx += 32 * kWarps) {
+                        const int r = rows + idx / (D / 8);
+                        *reinterpret_cast<uint4 *>(stage + stage_offset(r, idx % (D / 8))) = make_uint4(0, 0, 0, 0);
+                    }
+                    ptx::fence_proxy_async_smem();
+                    if (!gb.sync(sf)) { ok = false; break; }
+                }
+                const uint32_t sbase = ptx::smem_addr(stage);
+#pragma unroll
+                for (int kb = 0; kb < kSub; kb += 16) {
+                    // A operand: P of row gid for keys kb .. kb+15 (bf16), zero beyond RG
+                    uint32_t pa[4] = {0u, 0u, 0u, 0u};
+                    if (row_real) {
+                        const float2 p0 = *reinterpret_cast<const float2 *>(&s_sm[gid][t * kSub + kb + 2 * tig]);
+                        const float2 p1 = *reinterpret_cast<const float2 *>(&s_sm[gid][t * kSub + kb + 8 + 2 * tig]);
+                        pa[0] = pack2_bf16(p0.x, p0.y);
+                        pa[2] = pack2_bf16(p1.x, p1.y);
+                    }
+#pragma unroll
+                    for (int j = 0; j < NT; j += 2) {
+                        // matrices: (keys kb..+7 | kb+8..+15) x (column tile j | j+1)
+                        const int chunk = (warp * NT + j) + (lm_mat >> 1);
+                        const int row = kb + (lm_mat & 1) * 8 + lm_row;
+                        uint32_t b0, b1, b2, b3;
+                        ptx::ldsm_x4_trans(sbase + stage_offset(row, chunk), b0, b1, b2, b3);
+                        ptx::mma_16816_bf16(acc[j], pa, b0, b1);
+                        ptx::mma_16816_bf16(acc[j + 1], pa, b2, b3);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&empty[st]);
+                ++ring;
+            }
+            if (!ok) break;
+            const int chunk = start / kChunk;
+            if (row_real) {
+                const float inv_l = 1.f / l_sm[gid];
+                float *dst = p.part_o + (((size_t)b * p.Hq + h0 + gid) * p.S_max + chunk) * D;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    const int col = (warp * NT + j) * 8 + 2 * tig;
+                    *reinterpret_cast<float2 *>(dst + col) = make_float2(acc[j][0] * inv_l, acc[j][1] * inv_l);
+                }
+            }
+            if (threadIdx.x < RG)
+                p.part_lse[((size_t)b * p.Hq + h0 + threadIdx.x) * p.S_max + chunk] =
+                    m_sm[threadIdx.x] + ptx::lg2(l_sm[threadIdx.x]);
+            // scores and m/l are rewritten by the next item
+            if (!gb.sync(sf)) break;
+        }
     }
     __syncthreads();
-
-    for (int idx = threadIdx.x; idx < RG * D; idx += kThreads) {
-        const int r = idx / D;
-        const int e = idx - r * D;
-        float t = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) t += red[w][r][e];
-        p.part_o[(((size_t)b * p.Hq + h0 + r) * p.S_max + chunk) * D + e] = t / l_sm[r];
-    }
-    if (threadIdx.x < RG)
-        p.part_lse[((size_t)b * p.Hq + h0 + threadIdx.x) * p.S_max + chunk] =
-            m_sm[threadIdx.x] + ptx::lg2(l_sm[threadIdx.x]);
 }
 
 // One CTA of kMergeWarps warps per (query head, sequence).  Every warp finds the largest

@@ -23,7 +23,7 @@
 //   warps 0-3   softmax for Q tile 0, warps 4-7 for Q tile 1 (one thread per row):
 //               load S_s from TMEM, mask, row max, exp2 with the scale folded in
 //               (p = 2^(s*scale*log2e - m)), lazy rescale (the reference maximum is only
-//               moved when the new one exceeds it by more than 8 in log2 units; O_s is
+//               moved when the new one exceeds it by more than 16 in log2 units; O_s is
 //               then rescaled in TMEM by the same warp), P_s to TMEM as bf16, fp32 row
 //               sum; at the end of a unit O_s / l and LSE are written out.
 //   warps 10-11 idle (they complete the third warpgroup, which lends registers to the
@@ -74,7 +74,7 @@ constexpr int kRegsLow = 72;
 constexpr int kRegsHigh = 216;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch budget");
 constexpr int kChunkBytes = 128 * 128;  // one 64-column (128-byte) slab of a 128-row tile
-constexpr float kLazyThreshold = 8.0f;  // log2 units: rescale only past a factor of 256
+constexpr float kLazyThreshold = 16.0f;  // log2 units: rescale only past a factor of 2^16
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D>
@@ -87,8 +87,8 @@ struct Cfg {
     static constexpr int kKVOff = 4 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
     // barriers: kv_full[S], kv_empty[S], q_full[2 sets][2], q_empty[2 sets][2], s_full[2],
-    //           p_ready[2], o_done[2], o_free[2], teardown
-    static constexpr int kNumBars = 2 * kStages + 17;
+    //           p_ready[2], o_done[2], o_free[2], teardown, epilogue group[2]
+    static constexpr int kNumBars = 2 * kStages + 19;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 };
@@ -291,6 +291,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
     uint64_t *o_done = q_full + 12;
     uint64_t *o_free = q_full + 14;
     uint64_t *teardown = q_full + 16;
+    uint64_t *epi_group = q_full + 17;  // [2]: the four warps of a softmax warpgroup
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
     int *stop_flag = reinterpret_cast<int *>(smem + C::kMiscOff + 4);
 
@@ -315,6 +316,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             ptx::mbar_init(&o_free[s], 128);
         }
         ptx::mbar_init(teardown, 1);
+        ptx::mbar_init(&epi_group[0], 4);
+        ptx::mbar_init(&epi_group[1], 4);
         *stop_flag = 0;
         ptx::fence_barrier_init();
     }
@@ -525,6 +528,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         const uint32_t tS = tmem + lane_base + 128u * s;        // S_s, and P_s over it
         const uint32_t tO = tmem + lane_base + 256u + 128u * s;  // O_s
         const float sl2 = p.scale_log2;
+        GroupBarrier eg{&epi_group[s], 0u};
         uint32_t s_ph = 0, units = 0;
         Unit w;
         for (int u = next_unit(p, 2 * (int)blockIdx.x, w); u >= 0; u = next_unit(p, unit_step(u), w)) {
@@ -632,8 +636,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     *reinterpret_cast<uint4 *>(stage + slab * kChunkBytes + tid * 128 + chunk * 16) = v4;
                 }
                 ptx::fence_proxy_async_smem();
-                if (s == 0) ptx::named_barrier_sync<1, 128>();
-                else ptx::named_barrier_sync<2, 128>();
+                if (!eg.sync(sf)) break;
                 if (tid == 0) {
 #pragma unroll
                     for (int c = 0; c < D / 64; ++c)

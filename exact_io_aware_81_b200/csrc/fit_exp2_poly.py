@@ -6,7 +6,8 @@ scores).  The remaining coefficients minimise the maximum relative error
 |q(f) / 2^f - 1| on [-1/2, 1/2], found with Lawson's iteratively reweighted least squares
 (an approximation of the minimax/Remez solution) on a dense grid, in float64.
 
-Run:  python fit_exp2_poly.py [degree]   -- prints the coefficients c1..cn and the error.
+Run:  python fit_exp2_poly.py [degree]   -- prints the coefficients c1..cn and the error
+(the kernels use degree 4).
 """
 import sys
 
@@ -46,7 +47,7 @@ def max_error_float32(c):
 
 
 if __name__ == "__main__":
-    deg = int(sys.argv[1]) if len(sys.argv) > 1 else 3
+    deg = int(sys.argv[1]) if len(sys.argv) > 1 else 4
     c, err = fit(deg)
     for k, ck in enumerate(c, start=1):
         print(f"c{k} = {np.float32(ck)!r}  ({ck:.12e})")

@@ -81,6 +81,17 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// 1-D bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global
+// to shared memory; completion is counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
 // 3-D tiled store of one box from shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int x, int y, int z)
 {
@@ -216,6 +227,36 @@ __device__ __forceinline__ void regs_increase() { asm volatile("setmaxnreg.inc.s
 template <int N>
 __device__ __forceinline__ void regs_decrease() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
+// ------------------------------------------------- warp-level MMA (mma.sync) helpers
+
+// Four 8x8 b16 matrices from shared memory; lane i supplies row (i & 7) of matrix i >> 3.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr)
+                 : "memory");
+}
+
+// As ldsm_x4, each matrix transposed.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr)
+                 : "memory");
+}
+
+// D (16x8 fp32) += A (16x16 bf16, row-major fragment) * B (16x8 bf16, column fragment).
+__device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // ------------------------------------------------------------ matrix descriptors
 
 // Shared-memory matrix descriptor (tcgen05 format): start address, leading and stride
@@ -268,20 +309,22 @@ __device__ __forceinline__ float max3(float a, float b, float c)
 
 // 2^y for two lanes on the FMA pipe, for y <= 2^22 (masked -inf included): y is clamped to
 // >= -127, split as y = j + f with j = round(y) (by adding and subtracting 1.5 * 2^23) and
-// f in [-1/2, 1/2]; q(f) ~ 2^f is a degree-3 polynomial with q(0) = 1 whose coefficients
-// come from fit_exp2_poly.py (Lawson minimax fit, max relative error 1.0e-4, below the
-// 2^-9 rounding of the bf16 P it feeds); j is added to the exponent field of q(f).  At
-// y = -127 the result packs to exactly +0.
+// f in [-1/2, 1/2]; q(f) ~ 2^f is a degree-4 polynomial with q(0) = 1 whose coefficients
+// come from fit_exp2_poly.py 4 (Lawson minimax fit, max relative error 2.9e-6, far below
+// the 2^-9 rounding of the bf16 P it feeds, so it rounds to the same bf16 as the MUFU
+// result in all but rare cases); j is added to the exponent field of q(f).  At y = -127
+// the result packs to exactly +0.
 __device__ __forceinline__ float2 exp2_poly2(float2 y)
 {
     constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    constexpr float c1 = 0.69328296f, c2 = 0.24221097f, c3 = 0.055008568f;
+    constexpr float c1 = 0.6931242f, c2 = 0.24024099f, c3 = 0.055906463f, c4 = 0.009582838f;
     y.x = fmaxf(y.x, -127.0f);
     y.y = fmaxf(y.y, -127.0f);
     const float2 t = __fadd2_rn(y, make_float2(kRound, kRound));
     const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
     const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), y);
-    float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+    float2 q = __ffma2_rn(make_float2(c4, c4), f, make_float2(c3, c3));
+    q = __ffma2_rn(q, f, make_float2(c2, c2));
     q = __ffma2_rn(q, f, make_float2(c1, c1));
     q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
     return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),

@@ -1,9 +1,9 @@
 """The FMA-pipe exp2 used for a quarter of the softmax exponentials, checked against 2^x
 in float64 and against the hardware ex2 on the same inputs.
 
-The polynomial's stated bound (fit_exp2_poly.py: max relative error 1.0e-4 on the reduced
-argument) must hold over the whole range the softmax feeds it: x in [-127, 8], plus -inf
-for masked scores, which must give exactly +0.
+The polynomial's stated bound (fit_exp2_poly.py: max relative error 2.9e-6 (degree 4; 1.0e-4 at degree 3) on the reduced
+argument) must hold over the whole range the softmax feeds it: x in [-127, 16] (16 is the
+lazy-rescale threshold), plus -inf for masked scores, which must give exactly +0.
 """
 import ctypes
 import os
@@ -41,13 +41,13 @@ def run(lib, xs):
 
 
 def test_relative_error_over_softmax_range(probe):
-    xs = np.linspace(-126.0, 8.0, 1 << 20, dtype=np.float32)
+    xs = np.linspace(-126.0, 16.0, 1 << 20, dtype=np.float32)
     poly, mufu = run(probe, xs)
     exact = np.exp2(xs.astype(np.float64))
     rel = np.abs(poly / exact - 1.0)
-    assert rel.max() <= 1.1e-4, rel.max()
-    # no worse than 1.1e-4 relative to the hardware unit either
-    assert np.abs(poly / mufu - 1.0).max() <= 1.2e-4
+    assert rel.max() <= 4e-6, rel.max()
+    # and within 5e-6 of the hardware unit
+    assert np.abs(poly / mufu - 1.0).max() <= 5e-6
 
 
 def test_masked_and_underflow(probe):
@@ -58,7 +58,7 @@ def test_masked_and_underflow(probe):
 
 
 def test_integers_exact(probe):
-    xs = np.arange(-126, 9, dtype=np.float32)
+    xs = np.arange(-126, 17, dtype=np.float32)
     xs = np.concatenate([xs, xs[:1]])[: (len(xs) + 1) // 2 * 2]
     poly, _ = run(probe, xs)
     assert np.array_equal(poly, np.exp2(xs.astype(np.float64)))
