@@ -48,7 +48,7 @@ struct DeviceInfo {
     bool valid = false;
     bool sm100 = false;
     int num_sms = 0;
-    bool prefill_attr_set[2][2] = {{false, false}, {false, false}};
+    bool prefill_attr_set[2][2][2] = {};
     bool decode_attr_set[2][4] = {{false, false, false, false}, {false, false, false, false}};
 };
 constexpr int kMaxDevices = 64;
@@ -139,14 +139,14 @@ int validate_fwd(const void *q, const void *k, const void *v, const void *o, con
     return FA_OK;
 }
 
-template <int D, bool F32>
+template <int D, bool F32, bool SPLIT>
 int launch_prefill(const fa::PrefillParams &p, DeviceInfo *info, cudaStream_t st)
 {
     using C = fa::prefill::Cfg<D>;
-    auto kern = fa::fa_prefill_kernel<D, F32>;
+    auto kern = fa::fa_prefill_kernel<D, F32, SPLIT>;
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
-        bool &set = info->prefill_attr_set[D == 128][F32];
+        bool &set = info->prefill_attr_set[D == 128][F32][SPLIT];
         if (!set) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  C::kSmemBytes);
@@ -206,8 +206,13 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     p.selftest_no_s_signal = selftest_timeout;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (d == 128) rc = o_dtype == FA_F32 ? launch_prefill<128, true>(p, info, st) : launch_prefill<128, false>(p, info, st);
-    else rc = o_dtype == FA_F32 ? launch_prefill<64, true>(p, info, st) : launch_prefill<64, false>(p, info, st);
+    const bool f32 = o_dtype == FA_F32, split = p.head_pair != 0;
+    if (d == 128)
+        rc = f32 ? (split ? launch_prefill<128, true, true>(p, info, st) : launch_prefill<128, true, false>(p, info, st))
+                 : (split ? launch_prefill<128, false, true>(p, info, st) : launch_prefill<128, false, false>(p, info, st));
+    else
+        rc = f32 ? (split ? launch_prefill<64, true, true>(p, info, st) : launch_prefill<64, true, false>(p, info, st))
+                 : (split ? launch_prefill<64, false, true>(p, info, st) : launch_prefill<64, false, false>(p, info, st));
     if (rc != FA_OK) return rc;
     return ok();
 }

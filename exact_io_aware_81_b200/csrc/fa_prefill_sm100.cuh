@@ -87,8 +87,8 @@ struct Cfg {
     static constexpr int kKVOff = 4 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
     // barriers: kv_full[S], kv_empty[S], q_full[2 sets][2], q_empty[2 sets][2], s_full[2],
-    //           p_ready[2], o_done[2], o_free[2], teardown, epilogue group[2]
-    static constexpr int kNumBars = 2 * kStages + 19;
+    //           p_ready[2], o_done[2], o_free[2], teardown, epilogue group[2], p_half[2]
+    static constexpr int kNumBars = 2 * kStages + 21;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 };
@@ -174,18 +174,18 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_saddr, uint
     }
 }
 
-// O (+)= P V: 8 MMAs of K = 16 keys.  P (128 x 128 bf16) is read from tensor memory, 8
-// columns per K step.  V is an MN-major (d contiguous) 128-byte-swizzled tile: 8-key
+// O (+)= P V for K steps [k_begin, k_end) of the 8 (16 keys each).  P (128 x 128 bf16)
+// is read from tensor memory, 8 columns per K step.  V is an MN-major (d contiguous) 128-byte-swizzled tile: 8-key
 // groups 1024 bytes apart (stride offset), 64-column slabs of d 16 KB apart (leading
 // offset), and a K step of 16 keys advances 2048 bytes.
-template <int D>
+template <int D, int K_BEGIN, int K_END>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_saddr,
                                          bool accumulate)
 {
     constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, D, 1);
     const uint64_t b0 = ptx::smem_desc_sw128(v_saddr, kChunkBytes, 1024);
 #pragma unroll
-    for (int k = 0; k < BN / 16; ++k)
+    for (int k = K_BEGIN; k < K_END; ++k)
         ptx::mma_ts(d_tmem, p_tmem + k * 8, b0 + (uint64_t)(k * 2048 >> 4), idesc, (accumulate || k > 0) ? 1u : 0u);
 }
 
@@ -271,7 +271,9 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, uint6
 
 }  // namespace prefill
 
-template <int D, bool OUT_F32>
+// SPLIT_P: hand P to the MMA warp in two halves (used for head-pair units; measured to
+// help the grouped-query tiling and to cost a little on the row-pair tiling).
+template <int D, bool OUT_F32, bool SPLIT_P>
 __global__ void __launch_bounds__(prefill::kThreads, 1)
     fa_prefill_kernel(const __grid_constant__ PrefillParams p)
 {
@@ -292,6 +294,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
     uint64_t *o_free = q_full + 14;
     uint64_t *teardown = q_full + 16;
     uint64_t *epi_group = q_full + 17;  // [2]: the four warps of a softmax warpgroup
+    uint64_t *p_half = q_full + 19;     // [2]: first 64 keys of P_s written
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
     int *stop_flag = reinterpret_cast<int *>(smem + C::kMiscOff + 4);
 
@@ -312,6 +315,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             ptx::mbar_init(&q_empty[2 + s], 2);
             ptx::mbar_init(&s_full[s], 1);
             ptx::mbar_init(&p_ready[s], 128);
+            ptx::mbar_init(&p_half[s], 128);
             ptx::mbar_init(&o_done[s], 1);
             ptx::mbar_init(&o_free[s], 128);
         }
@@ -436,13 +440,34 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         // draining the tensor pipe at every unit.
         bool pend = false, pend_acc = false, pend_free = false;
         uint32_t pend_v = 0, pend_free_par = 0;
+        // P V of Q tile s.  With SPLIT_P in two halves: keys 0-63 as soon as the softmax
+        // has written that half of P, keys 64-127 when the whole tile is done.
+        auto issue_pv_halves = [&](int s, uint32_t v_stage, bool acc, bool need_free, uint32_t fpar) -> bool {
+            const uint32_t d_tmem = tmem + 256 + 128 * s, p_tmem = tmem + 128 * s;
+            const uint32_t v_saddr = kv_saddr0 + v_stage * C::kTileBytes;
+            if (SPLIT_P) {
+                if (need_free && !wait_warp(&o_free[s], fpar, sf)) return false;
+                if (!wait_warp(&p_half[s], p_ph[s], sf)) return false;
+                ptx::tc_fence_after();
+                if (leader) issue_pv<D, 0, 4>(d_tmem, p_tmem, v_saddr, acc);
+                __syncwarp();
+                if (!wait_warp(&p_ready[s], p_ph[s], sf)) return false;
+                p_ph[s] ^= 1u;
+                ptx::tc_fence_after();
+                if (leader) issue_pv<D, 4, 8>(d_tmem, p_tmem, v_saddr, true);
+            } else {
+                if (!wait_warp(&p_ready[s], p_ph[s], sf)) return false;
+                p_ph[s] ^= 1u;
+                if (need_free && !wait_warp(&o_free[s], fpar, sf)) return false;
+                ptx::tc_fence_after();
+                if (leader) issue_pv<D, 0, 8>(d_tmem, p_tmem, v_saddr, acc);
+            }
+            __syncwarp();
+            return true;
+        };
         auto issue_pv1 = [&](uint32_t v_stage, bool acc, bool need_free, uint32_t fpar, bool last) -> bool {
-            if (!wait_warp(&p_ready[1], p_ph[1], sf)) return false;
-            p_ph[1] ^= 1u;
-            if (need_free && !wait_warp(&o_free[1], fpar, sf)) return false;
-            ptx::tc_fence_after();
+            if (!issue_pv_halves(1, v_stage, acc, need_free, fpar)) return false;
             if (leader) {
-                issue_pv<D>(tmem + 384, tmem + 128, kv_saddr0 + v_stage * C::kTileBytes, acc);
                 ptx::mma_commit(&kv_empty[v_stage]);
                 if (last) ptx::mma_commit(&o_done[1]);
             }
@@ -491,14 +516,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 __syncwarp();
                 if (!wait_warp(&kv_full[vs], vph, sf)) { ok = false; break; }
                 if (j < w.n0) {
-                    if (!wait_warp(&p_ready[0], p_ph[0], sf)) { ok = false; break; }
-                    p_ph[0] ^= 1u;
-                    if (j == 0 && !wait_warp(&o_free[0], free_par, sf)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    if (leader) {
-                        issue_pv<D>(tmem + 256, tmem + 0, kv_saddr0 + vs * C::kTileBytes, j > 0);
-                        if (j == w.n0 - 1) ptx::mma_commit(&o_done[0]);
-                    }
+                    if (!issue_pv_halves(0, vs, j > 0, j == 0, free_par)) { ok = false; break; }
+                    if (leader && j == w.n0 - 1) ptx::mma_commit(&o_done[0]);
                     __syncwarp();
                 }
                 prev_v = vs;
@@ -568,22 +587,39 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     m = mx;
                     rescale = true;
                 }
-                sum = exp2_pack<64, 0, 0>(x, sl2, m) + exp2_pack<64, 64, 32>(x, sl2, m);
-                ptx::tmem_st32(tS + 0, &x[0]);
-                ptx::tmem_st32(tS + 32, &x[32]);
-                // Rare (lazy) rescale of the partial output, before P V of this tile is
-                // issued; warp-uniform because TMEM loads and stores are warp-collective.
-                if (__any_sync(0xffffffffu, rescale)) {
+                // Rare (lazy) rescale of the partial output, before any P V of this tile is
+                // issued (P V of the previous tile is complete: the commit that signalled
+                // this S tile covers it); warp-uniform because TMEM accesses are collective.
+                auto rescale_o = [&]() {
+                    if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t ov[32];
-                        ptx::tmem_ld32(tO + 32 * c, ov);
-                        ptx::tmem_wait_ld();
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t ov[32];
+                            ptx::tmem_ld32(tO + 32 * c, ov);
+                            ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                        ptx::tmem_st32(tO + 32 * c, ov);
+                            for (int e = 0; e < 32; ++e)
+                                ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                            ptx::tmem_st32(tO + 32 * c, ov);
+                        }
                     }
+                };
+                if (SPLIT_P) {
+                    // the first 64 keys of P are handed to the MMA warp while the second
+                    // half is still being computed
+                    rescale_o();
+                    sum = exp2_pack<64, 0, 0>(x, sl2, m);
+                    ptx::tmem_st32(tS + 0, &x[0]);
+                    ptx::tmem_wait_st();
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive(&p_half[s]);
+                    sum += exp2_pack<64, 64, 32>(x, sl2, m);
+                    ptx::tmem_st32(tS + 32, &x[32]);
+                } else {
+                    sum = exp2_pack<64, 0, 0>(x, sl2, m) + exp2_pack<64, 64, 32>(x, sl2, m);
+                    ptx::tmem_st32(tS + 0, &x[0]);
+                    ptx::tmem_st32(tS + 32, &x[32]);
+                    rescale_o();
                 }
                 ptx::tmem_wait_st();
                 const float p_top = ptx::ex2(mx - m);  // the tile's largest weight (0 if masked)
