@@ -41,22 +41,27 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def declare(lib):
+    """Set the ctypes signatures of the oracle's C entry points on a loaded library."""
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    D = ctypes.c_double
+    lib.oracle_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I, D, I, P, I, P, P]
+    lib.oracle_attn_fwd_window.argtypes = [P, P, P, I, I, I, I, I, I, D, I, I, P, I, P, P]
+    lib.oracle_attn_probs.argtypes = [P, P, I, I, I, I, I, I, D, I, P]
+    lib.oracle_attn_probs_window.argtypes = [P, P, I, I, I, I, I, I, D, I, I, P]
+    lib.oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, D, P, P]
+    lib.oracle_num_threads.argtypes = []
+    for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_window, lib.oracle_attn_probs,
+              lib.oracle_attn_probs_window, lib.oracle_decode, lib.oracle_num_threads):
+        f.restype = I
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        P = ctypes.c_void_p
-        I = ctypes.c_int
-        D = ctypes.c_double
-        lib.oracle_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I, D, I, P, I, P, P]
-        lib.oracle_attn_fwd.restype = I
-        lib.oracle_attn_probs.argtypes = [P, P, I, I, I, I, I, I, D, I, P]
-        lib.oracle_attn_probs.restype = I
-        lib.oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, D, P, P]
-        lib.oracle_decode.restype = I
-        lib.oracle_num_threads.argtypes = []
-        lib.oracle_num_threads.restype = I
-        _lib = lib
+        _lib = declare(ctypes.CDLL(build()))
     return _lib
 
 
@@ -74,9 +79,11 @@ def num_threads() -> int:
 
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float, causal: bool,
-             rows: Optional[torch.Tensor] = None):
+             rows: Optional[torch.Tensor] = None, window: int = 0):
     """fp64 attention of bf16 q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d).
 
+    ``window`` = W >= 1 restricts causal row i to its W most recent keys
+    (i + Nk - Nq - W < j <= i + Nk - Nq); 0 means no window.
     Returns (o, lse) as float64 torch tensors of shape (B,Hq,R,d) and (B,Hq,R), where R
     is len(rows) if a row sample is given, else Nq.
     """
@@ -91,20 +98,32 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float, ca
         rw, nr, rp = None, Nq, None
     o = np.empty((B, Hq, nr, d), dtype=np.float64)
     lse = np.empty((B, Hq, nr), dtype=np.float64)
-    rc = _load().oracle_attn_fwd(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Nq, Nk, d,
+    lib = _load()
+    if window:
+        rc = lib.oracle_attn_fwd_window(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Nq, Nk, d,
+                                        float(scale), int(bool(causal)), int(window), rp, nr,
+                                        _ptr(o), _ptr(lse))
+    else:
+        rc = lib.oracle_attn_fwd(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Nq, Nk, d,
                                  float(scale), int(bool(causal)), rp, nr, _ptr(o), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_attn_fwd rejected its arguments")
     return torch.from_numpy(o), torch.from_numpy(lse)
 
 
-def probs(q: torch.Tensor, k: torch.Tensor, scale: float, causal: bool) -> torch.Tensor:
-    """Softmax weights P (B,Hq,Nq,Nk) in fp64, for tiny problems."""
+def probs(q: torch.Tensor, k: torch.Tensor, scale: float, causal: bool,
+          window: int = 0) -> torch.Tensor:
+    """Softmax weights P (B,Hq,Nq,Nk) in fp64, for tiny problems (window as in attn_fwd)."""
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
     qb, kb = _bits(q), _bits(k)
     p = np.empty((B, Hq, Nq, Nk), dtype=np.float64)
-    rc = _load().oracle_attn_probs(_ptr(qb), _ptr(kb), B, Hq, Hkv, Nq, Nk, d, float(scale),
+    lib = _load()
+    if window:
+        rc = lib.oracle_attn_probs_window(_ptr(qb), _ptr(kb), B, Hq, Hkv, Nq, Nk, d,
+                                          float(scale), int(bool(causal)), int(window), _ptr(p))
+    else:
+        rc = lib.oracle_attn_probs(_ptr(qb), _ptr(kb), B, Hq, Hkv, Nq, Nk, d, float(scale),
                                    int(bool(causal)), _ptr(p))
     if rc != 0:
         raise ValueError("oracle_attn_probs rejected its arguments")

@@ -22,7 +22,12 @@
  *   - causal with Nq != Nk is bottom-right aligned: row i sees keys j <= i + Nk - Nq;
  *   - decode (one query row per sequence) sees every cached key j < L_b, unmasked;
  *   - lse is the natural log of sum_j exp(s_ij), scale included;
- *   - a row that sees no key (only L_b = 0 in decode) gives o = 0 and lse = -inf.
+ *   - a row that sees no key (only L_b = 0 in decode) gives o = 0 and lse = -inf;
+ *   - sliding window W (youngju.dev section 4: each token looks only at the W most
+ *     recent tokens, itself included -- with W = 3, query 5 sees keys 3, 4, 5) is a
+ *     lower bound on top of the causal limit: row i sees keys j with
+ *     i + Nk - Nq - W < j <= i + Nk - Nq.  It is defined for causal attention only;
+ *     W = 0 means no window.
  *
  * Parallelism: OpenMP over independent (batch, head, row) triples; each row is
  * computed start to finish by one thread, so the result does not depend on the
@@ -49,6 +54,15 @@ static long visible_keys(long i, long Nq, long Nk, int causal)
     long last = i + (Nk - Nq);          /* bottom-right aligned causal limit */
     if (last >= Nk) last = Nk - 1;
     return last < 0 ? 0 : last + 1;
+}
+
+/* First key that query row i may see: the sliding window's lower bound (0 without one).
+ * The keys row i sees are first_key(...) .. visible_keys(...) - 1. */
+static long first_key(long i, long Nq, long Nk, long window)
+{
+    if (window <= 0) return 0;
+    long first = i + (Nk - Nq) - window + 1;
+    return first > 0 ? first : 0;
 }
 
 /* One query row against keys [0, nkeys) of one K/V head; writes d outputs and lse. */
@@ -87,15 +101,17 @@ static void attend_row(const uint16_t *qrow, const uint16_t *khead, const uint16
  *   rows: optional list of nrows query-row indices applied to every (b, h); NULL means
  *         all Nq rows (nrows is then ignored).
  *   o: (B,Hq,R,d) doubles, lse: (B,Hq,R) doubles, R = nrows or Nq.
+ *   window: sliding-window width W >= 1 (causal only), or 0 for none.
  * Returns 0, or -1 on an argument error.
  */
-int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                    int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                    double scale, int causal, const int32_t *rows, int nrows,
-                    double *o, double *lse)
+int oracle_attn_fwd_window(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                           double scale, int causal, int window,
+                           const int32_t *rows, int nrows, double *o, double *lse)
 {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return -1;
     if (Hq % Hkv != 0) return -1;
+    if (window < 0 || (window > 0 && !causal)) return -1;
     const long R = Hq / Hkv;
     const long nr = rows ? nrows : Nq;
     const long total = (long)B * Hq * nr;
@@ -120,7 +136,9 @@ int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 const uint16_t *qrow = q + (((long)b * Hq + h) * Nq + i) * d;
                 const uint16_t *kh = k + ((long)b * Hkv + g) * (long)Nk * d;
                 const uint16_t *vh = v + ((long)b * Hkv + g) * (long)Nk * d;
-                attend_row(qrow, kh, vh, visible_keys(i, Nq, Nk, causal), d, scale,
+                long j0 = first_key(i, Nq, Nk, window);
+                long j1 = visible_keys(i, Nq, Nk, causal);
+                attend_row(qrow, kh + j0 * d, vh + j0 * d, j1 > j0 ? j1 - j0 : 0, d, scale,
                            qbuf, s, o + idx * d, lse + idx);
             }
         }
@@ -130,16 +148,27 @@ int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     return err ? -1 : 0;
 }
 
+/* The forward without a sliding window. */
+int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                    int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                    double scale, int causal, const int32_t *rows, int nrows,
+                    double *o, double *lse)
+{
+    return oracle_attn_fwd_window(q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0,
+                                  rows, nrows, o, lse);
+}
+
 /*
  * Softmax weights P (B,Hq,Nq,Nk) for tiny problems, by the same two passes; masked
  * entries are exactly 0.  Used only to check that each row of P sums to one.
  */
-int oracle_attn_probs(const uint16_t *q, const uint16_t *k,
-                      int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                      double scale, int causal, double *p)
+int oracle_attn_probs_window(const uint16_t *q, const uint16_t *k,
+                             int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                             double scale, int causal, int window, double *p)
 {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return -1;
     if (Hq % Hkv != 0) return -1;
+    if (window < 0 || (window > 0 && !causal)) return -1;
     const long R = Hq / Hkv;
     for (long b = 0; b < B; ++b)
         for (long h = 0; h < Hq; ++h)
@@ -148,11 +177,12 @@ int oracle_attn_probs(const uint16_t *q, const uint16_t *k,
                 const uint16_t *qrow = q + ((b * Hq + h) * Nq + i) * d;
                 const uint16_t *kh = k + (b * Hkv + g) * (long)Nk * d;
                 double *prow = p + ((b * Hq + h) * Nq + i) * (long)Nk;
+                long j0 = first_key(i, Nq, Nk, window);
                 long nk = visible_keys(i, Nq, Nk, causal);
                 for (long j = 0; j < Nk; ++j) prow[j] = 0.0;
-                if (nk <= 0) continue;
+                if (nk <= j0) continue;
                 double m = -INFINITY;
-                for (long j = 0; j < nk; ++j) {
+                for (long j = j0; j < nk; ++j) {
                     double acc = 0.0;
                     for (long t = 0; t < d; ++t)
                         acc += bf16_bits_to_double(qrow[t]) * bf16_bits_to_double(kh[j * d + t]);
@@ -160,10 +190,18 @@ int oracle_attn_probs(const uint16_t *q, const uint16_t *k,
                     if (prow[j] > m) m = prow[j];
                 }
                 double l = 0.0;
-                for (long j = 0; j < nk; ++j) l += exp(prow[j] - m);
-                for (long j = 0; j < nk; ++j) prow[j] = exp(prow[j] - m) / l;
+                for (long j = j0; j < nk; ++j) l += exp(prow[j] - m);
+                for (long j = j0; j < nk; ++j) prow[j] = exp(prow[j] - m) / l;
             }
     return 0;
+}
+
+/* The weights without a sliding window. */
+int oracle_attn_probs(const uint16_t *q, const uint16_t *k,
+                      int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                      double scale, int causal, double *p)
+{
+    return oracle_attn_probs_window(q, k, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, p);
 }
 
 /*

@@ -35,8 +35,9 @@ def _rand(shape, seed, std=1.0):
     return _bf16(torch.randn(shape, generator=g) * std)
 
 
-def _sdpa_ref(q, k, v, scale, causal):
-    """torch CPU fp64 SDPA with a bottom-right causal mask and GQA expansion."""
+def _sdpa_ref(q, k, v, scale, causal, window=0):
+    """torch CPU fp64 SDPA with a bottom-right causal mask (optionally banded to the W most
+    recent keys) and GQA expansion."""
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
     R = Hq // Hkv
@@ -48,6 +49,8 @@ def _sdpa_ref(q, k, v, scale, causal):
         i = torch.arange(Nq).view(-1, 1)
         j = torch.arange(Nk).view(1, -1)
         mask = j <= i + (Nk - Nq)
+        if window:
+            mask = mask & (j > i + (Nk - Nq) - window)
     o = F.scaled_dot_product_attention(qd, kd, vd, attn_mask=mask, scale=scale)
     s = torch.matmul(qd, kd.transpose(-1, -2)) * scale
     if mask is not None:
@@ -259,6 +262,52 @@ def pin_row_sample_matches_full():
     assert torch.equal(o[:, :, rows.long()], os_) and torch.equal(l[:, :, rows.long()], ls)
 
 
+def pin_sliding_window_golden():
+    """The page's W = 3 example: exactly the listed keys get weight, and they sum to one."""
+    rows = [list(map(int, ln.split())) for ln in open(os.path.join(GOLDEN, "sliding_window_w3.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    N = 8
+    q = _rand((1, 1, N, 8), 40)
+    k = _rand((1, 1, N, 8), 41)
+    p = oracle.probs(q, k, 0.5, True, window=3)[0, 0]
+    for row in rows:
+        i, keys = row[0], row[1:]
+        assert torch.nonzero(p[i]).flatten().tolist() == keys, (i, keys)
+        assert abs(p[i].sum().item() - 1.0) < 1e-12
+
+
+def pin_sliding_window_library_sdpa():
+    """Band-masked torch fp64 SDPA, square and chunked (Nq < Nk), MHA and GQA."""
+    for (Hq, Hkv, Nq, Nk, W, seed) in [(2, 2, 37, 37, 5, 42), (4, 2, 23, 61, 9, 45),
+                                       (4, 1, 50, 50, 1, 48), (2, 1, 17, 40, 64, 51)]:
+        q = _rand((2, Hq, Nq, 16), seed)
+        k = _rand((2, Hkv, Nk, 16), seed + 1)
+        v = _rand((2, Hkv, Nk, 16), seed + 2)
+        o, lse = oracle.attn_fwd(q, k, v, 0.3, True, window=W)
+        ro, rl = _sdpa_ref(q, k, v, 0.3, True, window=W)
+        assert torch.allclose(o, ro, atol=1e-12, rtol=0), (Hq, Hkv, Nq, Nk, W)
+        assert torch.allclose(lse, rl, atol=1e-12, rtol=0), (Hq, Hkv, Nq, Nk, W)
+
+
+def pin_window_special_cases():
+    """W >= Nk is plain causal; W = 1 picks the diagonal key: o_i = v[i + Nk - Nq] and
+    lse_i = scale * q_i . k_(i + Nk - Nq), by hand."""
+    Nq, Nk, d = 9, 14, 8
+    q = _rand((1, 2, Nq, d), 54)
+    k = _rand((1, 1, Nk, d), 55)
+    v = _rand((1, 1, Nk, d), 56)
+    oc, lc = oracle.attn_fwd(q, k, v, 0.7, True)
+    ow, lw = oracle.attn_fwd(q, k, v, 0.7, True, window=Nk)
+    assert torch.equal(oc, ow) and torch.equal(lc, lw)
+    o1, l1 = oracle.attn_fwd(q, k, v, 0.7, True, window=1)
+    for h in range(2):
+        for i in range(Nq):
+            j = i + Nk - Nq
+            assert torch.equal(o1[0, h, i], v[0, 0, j].double())
+            dot = sum(float(q[0, h, i, t]) * float(k[0, 0, j, t]) for t in range(d))
+            assert abs(l1[0, h, i].item() - 0.7 * dot) < 1e-12
+
+
 PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]
 
 
@@ -280,6 +329,8 @@ MUTANTS = [
     ("transposed k index", "const uint16_t *kr = khead + j * d;", "const uint16_t *kr = khead + j;"),
     ("normaliser dropped", "double p = exp(s[j] - m) / l;", "double p = exp(s[j] - m);"),
     ("last key dropped", "for (long j = 0; j < nkeys; ++j) {\n        double p", "for (long j = 0; j + 1 < nkeys; ++j) {\n        double p"),
+    ("window off by one", "long first = i + (Nk - Nq) - window + 1;", "long first = i + (Nk - Nq) - window;"),
+    ("window offset dropped", "long first = i + (Nk - Nq) - window + 1;", "long first = i - window + 1;"),
 ]
 
 
@@ -294,11 +345,7 @@ def test_pins_catch_planted_mistake(name, old, new, monkeypatch):
         open(c, "w").write(mutated)
         subprocess.check_call(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", so, c, "-lm"])
         import ctypes
-        lib = ctypes.CDLL(so)
-        P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
-        lib.oracle_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I, D, I, P, I, P, P]
-        lib.oracle_attn_probs.argtypes = [P, P, I, I, I, I, I, I, D, I, P]
-        lib.oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, D, P, P]
+        lib = oracle.declare(ctypes.CDLL(so))
         monkeypatch.setattr(oracle, "_lib", lib)
         caught = []
         for pin in PINS:
