@@ -48,7 +48,7 @@ struct DeviceInfo {
     bool valid = false;
     bool sm100 = false;
     int num_sms = 0;
-    bool prefill_attr_set[2][2][2] = {};
+    bool prefill_attr_set[2][2][2][2] = {};
     bool decode_attr_set[2][4] = {{false, false, false, false}, {false, false, false, false}};
 };
 constexpr int kMaxDevices = 64;
@@ -139,14 +139,14 @@ int validate_fwd(const void *q, const void *k, const void *v, const void *o, con
     return FA_OK;
 }
 
-template <int D, bool F32, bool SPLIT>
+template <int D, bool F32, bool SPLIT, bool WINDOW>
 int launch_prefill(const fa::PrefillParams &p, DeviceInfo *info, cudaStream_t st)
 {
     using C = fa::prefill::Cfg<D>;
-    auto kern = fa::fa_prefill_kernel<D, F32, SPLIT>;
+    auto kern = fa::fa_prefill_kernel<D, F32, SPLIT, WINDOW>;
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
-        bool &set = info->prefill_attr_set[D == 128][F32][SPLIT];
+        bool &set = info->prefill_attr_set[D == 128][F32][SPLIT][WINDOW];
         if (!set) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  C::kSmemBytes);
@@ -162,12 +162,25 @@ int launch_prefill(const fa::PrefillParams &p, DeviceInfo *info, cudaStream_t st
     return FA_OK;
 }
 
+// Kernel variant for one head dim and output type: P handed over in halves for head-pair
+// tiling, and the sliding-window variant only when a window is set.
+template <int D, bool F32>
+int launch_prefill_variant(const fa::PrefillParams &p, DeviceInfo *info, cudaStream_t st)
+{
+    const bool win = p.window > 0;
+    if (p.head_pair)
+        return win ? launch_prefill<D, F32, true, true>(p, info, st) : launch_prefill<D, F32, true, false>(p, info, st);
+    return win ? launch_prefill<D, F32, false, true>(p, info, st) : launch_prefill<D, F32, false, false>(p, info, st);
+}
+
 int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
-             int Hkv, int Nq, int Nk, int d, float scale, int causal, int o_dtype, void *stream,
-             int selftest_timeout)
+             int Hkv, int Nq, int Nk, int d, float scale, int causal, int window, int o_dtype,
+             void *stream, int selftest_timeout)
 {
     int rc = validate_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, o_dtype);
     if (rc != FA_OK) return rc;
+    if (window < 0) return fail(FA_ERR_INVALID, "window must be >= 0 (got %d)", window);
+    if (window > 0 && !causal) return fail(FA_ERR_INVALID, "a sliding window needs causal attention");
     int dev;
     DeviceInfo *info;
     if ((rc = current_device(&dev, &info)) != FA_OK) return rc;
@@ -187,6 +200,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     p.Nk = Nk;
     p.R = Hq / Hkv;
     p.causal = causal ? 1 : 0;
+    p.window = window < Nk ? window : 0;  // a window of Nk or more keys is plain causal
     p.head_pair = (p.R % 2 == 0) ? 1 : 0;
     const int tiles = (Nq + 127) / 128;
     long long head_slots;
@@ -206,13 +220,11 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     p.selftest_no_s_signal = selftest_timeout;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool f32 = o_dtype == FA_F32, split = p.head_pair != 0;
+    const bool f32 = o_dtype == FA_F32;
     if (d == 128)
-        rc = f32 ? (split ? launch_prefill<128, true, true>(p, info, st) : launch_prefill<128, true, false>(p, info, st))
-                 : (split ? launch_prefill<128, false, true>(p, info, st) : launch_prefill<128, false, false>(p, info, st));
+        rc = f32 ? launch_prefill_variant<128, true>(p, info, st) : launch_prefill_variant<128, false>(p, info, st);
     else
-        rc = f32 ? (split ? launch_prefill<64, true, true>(p, info, st) : launch_prefill<64, true, false>(p, info, st))
-                 : (split ? launch_prefill<64, false, true>(p, info, st) : launch_prefill<64, false, false>(p, info, st));
+        rc = f32 ? launch_prefill_variant<64, true>(p, info, st) : launch_prefill_variant<64, false>(p, info, st);
     if (rc != FA_OK) return rc;
     return ok();
 }
@@ -291,20 +303,28 @@ extern "C" {
 int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
            int Hkv, int Nq, int Nk, int d, float scale, int causal, void *stream)
 {
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, FA_BF16, stream, 0);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, stream, 0);
 }
 
 int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
               int Hkv, int Nq, int Nk, int d, float scale, int causal, int o_dtype, void *stream)
 {
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, o_dtype, stream, 0);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, o_dtype, stream, 0);
+}
+
+int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                  int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window, int o_dtype,
+                  void *stream)
+{
+    if (window <= 0) return fail(FA_ERR_INVALID, "window must be >= 1 (got %d)", window);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, o_dtype, stream, 0);
 }
 
 int fa_fwd_selftest_timeout(const void *q, const void *k, const void *v, void *o, float *lse,
                             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
                             int causal, void *stream)
 {
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, FA_BF16, stream, 1);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, stream, 1);
 }
 
 size_t fa_decode_workspace_size(int B, int Hq, int Nmax, int d) { return decode_ws_bytes(B, Hq, Nmax, d); }

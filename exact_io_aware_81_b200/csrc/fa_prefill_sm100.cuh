@@ -53,6 +53,7 @@ struct PrefillParams {
     int B, Hq, Hkv, Nq, Nk;
     int R;           // Hq / Hkv
     int causal;
+    int window;      // sliding window W (causal only): row i sees keys (i+Nk-Nq-W, i+Nk-Nq]; 0 = none
     int head_pair;   // 1: a unit = heads (2p, 2p+1) of one group on the same 128 rows
     int T;           // tile rows per head slot: 128-row tiles (head_pair) or 256-row pairs
     int P;           // slots per head slot: ceil(T/2) if causal (units paired), else T
@@ -93,8 +94,11 @@ struct Cfg {
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 };
 
+// A unit: two 128-row Q tiles (s = 0, 1) of one K/V group; tile s reads key tiles
+// [a_s, n_s).  a0 <= a1 and n0 <= n1, and every key tile in [a0, n1) is read by at least
+// one of the two.
 struct Unit {
-    int b, g, h0, h1, r0, r1, n0, n1;
+    int b, g, h0, h1, r0, r1, a0, a1, n0, n1;
 };
 
 // Work is dealt out in slots.  A slot belongs to one "head slot" (a head pair of one
@@ -105,6 +109,9 @@ struct Unit {
 // running at any moment share few K/V heads and their tiles are re-read from L2.
 __device__ __forceinline__ int units_in_slot(const PrefillParams &p) { return p.causal ? 2 : 1; }
 
+// WINDOW: the kernel variant for sliding-window attention (p.window > 0); without it
+// a0 = a1 = 0 are compile-time constants and the plain causal code is unchanged.
+template <bool WINDOW>
 __device__ __forceinline__ bool decode_unit(const PrefillParams &p, int slot, int k, Unit &w)
 {
     const int hh = slot / p.P;
@@ -132,11 +139,22 @@ __device__ __forceinline__ bool decode_unit(const PrefillParams &p, int slot, in
         w.r1 = w.r0 + BM;
     }
     const int nkt = (p.Nk + BN - 1) / BN;
+    w.a0 = w.a1 = 0;
     if (p.causal) {
         const int delta = p.Nk - p.Nq;
         // the last row of a tile, r + 127, sees keys up to r + 127 + delta
         w.n0 = min(nkt, (w.r0 + BM - 1 + delta) / BN + 1);
         w.n1 = min(nkt, (w.r1 + BM - 1 + delta) / BN + 1);
+        if (WINDOW) {
+            // the first row of a tile, r, sees keys from r + delta - W + 1 on
+            w.a0 = max(0, w.r0 + delta - p.window + 1) / BN;
+            w.a1 = max(0, w.r1 + delta - p.window + 1) / BN;
+            // The second tile of a row pair can lie wholly past Nq (odd tile count) and
+            // then past every window: its rows are never stored, so it reads only the
+            // last key tile.  (Every other tile has a_s < n_s: its first row sees at
+            // least its own diagonal key.)
+            if (w.r1 >= p.Nq) w.a1 = w.n1 - 1;
+        }
     } else {
         w.n0 = w.n1 = nkt;
     }
@@ -148,10 +166,11 @@ __device__ __forceinline__ bool decode_unit(const PrefillParams &p, int slot, in
 __device__ __forceinline__ int unit_step(int u) { return u + ((u & 1) ? 2 * (int)gridDim.x - 1 : 1); }
 
 // First valid unit index >= u of this CTA (decoded into w), or -1.
+template <bool WINDOW>
 __device__ __forceinline__ int next_unit(const PrefillParams &p, int u, Unit &w)
 {
     for (; u < 2 * p.n_slots; u = unit_step(u))
-        if ((u & 1) < units_in_slot(p) && decode_unit(p, u >> 1, u & 1, w)) return u;
+        if ((u & 1) < units_in_slot(p) && decode_unit<WINDOW>(p, u >> 1, u & 1, w)) return u;
     return -1;
 }
 
@@ -255,6 +274,17 @@ __device__ __forceinline__ void mask_cols(uint32_t (&x)[128], int kbase, int lim
     }
 }
 
+// Set scores of keys before this row's first visible key (sliding window) to -inf.
+template <int C0, int NC>
+__device__ __forceinline__ void mask_cols_below(uint32_t (&x)[128], int kbase, int first)
+{
+    if (kbase + C0 < first) {
+#pragma unroll
+        for (int c = C0; c < C0 + NC; ++c)
+            if (kbase + c < first) x[c] = __float_as_uint(-INFINITY);
+    }
+}
+
 // A wait that ignores the stop flag, used only to let copies and MMAs already in
 // flight finish before the CTA leaves.
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
@@ -273,7 +303,7 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, uint6
 
 // SPLIT_P: hand P to the MMA warp in two halves (used for head-pair units; measured to
 // help the grouped-query tiling and to cost a little on the row-pair tiling).
-template <int D, bool OUT_F32, bool SPLIT_P>
+template <int D, bool OUT_F32, bool SPLIT_P, bool WINDOW>
 __global__ void __launch_bounds__(prefill::kThreads, 1)
     fa_prefill_kernel(const __grid_constant__ PrefillParams p)
 {
@@ -374,17 +404,17 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         auto q_slot = [&](uint32_t i, int s) { return &q_empty[2 * (int)(i & 1u) + s]; };
         auto q_free_parity = [&](uint32_t i) { return ((i >> 1) & 1u) ^ 1u; };
         Unit w, wn;
-        int u = next_unit(p, 2 * (int)blockIdx.x, w);
+        int u = next_unit<WINDOW>(p, 2 * (int)blockIdx.x, w);
         uint32_t i = 0;
         for (int s = 0; ok && u >= 0 && s < 2; ++s) {
             if (!wait_warp(q_slot(0, s), q_free_parity(0), sf)) ok = false;
             else issue_q(w, 0, s);
         }
         for (; ok && u >= 0; ++i) {
-            const int un = next_unit(p, unit_step(u), wn);
+            const int un = next_unit<WINDOW>(p, unit_step(u), wn);
             int q_next = (un >= 0) ? 0 : 2;  // look-ahead Q tiles already issued
             const int plane = w.b * p.Hkv + w.g;
-            for (int j = 0; j < w.n1 && ok; ++j) {
+            for (int j = w.a0; j < w.n1 && ok; ++j) {
                 for (int kv = 0; kv < 2; ++kv) {
                     const uint32_t st = kv_it % C::kStages;
                     const uint32_t ph = (kv_it / C::kStages) & 1u;
@@ -475,7 +505,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             return true;
         };
         Unit w;
-        for (int u = next_unit(p, 2 * (int)blockIdx.x, w); ok && u >= 0; u = next_unit(p, unit_step(u), w)) {
+        for (int u = next_unit<WINDOW>(p, 2 * (int)blockIdx.x, w); ok && u >= 0; u = next_unit<WINDOW>(p, unit_step(u), w)) {
             const uint32_t free_par = (units & 1u) ^ 1u;  // first unit passes at once
             const uint32_t qset = units & 1u;
             const uint32_t q_par = (units >> 1) & 1u;
@@ -485,7 +515,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             if (!wait_warp(&qf[0], q_par, sf) || !wait_warp(&qf[1], q_par, sf)) break;
             ptx::tc_fence_after();
             uint32_t prev_v = 0;
-            for (int j = 0; j < w.n1; ++j) {
+            // Key tile j feeds S0 / P V0 when a0 <= j < n0 and S1 / P V1 when a1 <= j < n1.
+            for (int j = w.a0; j < w.n1; ++j) {
                 const uint32_t ks = kv_it % C::kStages;
                 const uint32_t kph = (kv_it / C::kStages) & 1u;
                 const uint32_t vs = (kv_it + 1) % C::kStages;
@@ -501,23 +532,30 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     }
                     __syncwarp();
                 }
-                if (j > 0) {
-                    if (!issue_pv1(prev_v, j - 1 > 0, j - 1 == 0, free_par, false)) { ok = false; break; }
+                if (j > w.a1) {
+                    if (!issue_pv1(prev_v, j - 1 > w.a1, j - 1 == w.a1, free_par, false)) { ok = false; break; }
                 } else if (pend) {
                     if (!issue_pv1(pend_v, pend_acc, pend_free, pend_free_par, true)) { ok = false; break; }
                     pend = false;
                 }
                 if (leader) {
-                    issue_qk<D>(tmem + 128, q_saddr + C::kTileBytes, k_saddr);
-                    if (signal_s) ptx::mma_commit(&s_full[1]);
+                    if (j >= w.a1) {
+                        issue_qk<D>(tmem + 128, q_saddr + C::kTileBytes, k_saddr);
+                        if (signal_s) ptx::mma_commit(&s_full[1]);
+                    }
                     ptx::mma_commit(&kv_empty[ks]);
                     if (j == w.n1 - 1) ptx::mma_commit(&qe[1]);
                 }
                 __syncwarp();
                 if (!wait_warp(&kv_full[vs], vph, sf)) { ok = false; break; }
                 if (j < w.n0) {
-                    if (!issue_pv_halves(0, vs, j > 0, j == 0, free_par)) { ok = false; break; }
+                    if (!issue_pv_halves(0, vs, j > w.a0, j == w.a0, free_par)) { ok = false; break; }
                     if (leader && j == w.n0 - 1) ptx::mma_commit(&o_done[0]);
+                    __syncwarp();
+                }
+                // a V tile that Q tile 1 never reads is released here (sliding window)
+                if (j < w.a1) {
+                    if (leader) ptx::mma_commit(&kv_empty[vs]);
                     __syncwarp();
                 }
                 prev_v = vs;
@@ -526,8 +564,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             if (!ok) break;
             pend = true;
             pend_v = prev_v;
-            pend_acc = w.n1 > 1;
-            pend_free = w.n1 == 1;
+            pend_acc = w.n1 - 1 > w.a1;
+            pend_free = w.n1 - 1 == w.a1;
             pend_free_par = free_par;
             ++units;
         }
@@ -550,19 +588,21 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         GroupBarrier eg{&epi_group[s], 0u};
         uint32_t s_ph = 0, units = 0;
         Unit w;
-        for (int u = next_unit(p, 2 * (int)blockIdx.x, w); u >= 0; u = next_unit(p, unit_step(u), w)) {
+        for (int u = next_unit<WINDOW>(p, 2 * (int)blockIdx.x, w); u >= 0; u = next_unit<WINDOW>(p, unit_step(u), w)) {
             const int h = s ? w.h1 : w.h0;
             const int r0 = s ? w.r1 : w.r0;
+            const int a = s ? w.a1 : w.a0;
             const int n = s ? w.n1 : w.n0;
             const int row = r0 + tid;
             const int lim = p.causal ? min(row + (p.Nk - p.Nq), p.Nk - 1) : p.Nk - 1;
+            const int first = WINDOW ? row + (p.Nk - p.Nq) - p.window + 1 : 0;
             // l: sum of the fp32 weights (gives the LSE).  lo: normaliser of O, the same sum
             // corrected, tile by tile, by the bf16 rounding of the tile's largest weight --
             // the rounding the P V product actually saw.  For a row dominated by one key
             // this makes O exactly that key's value row, as it should be.
             float m = -INFINITY, l = 0.f, lo = 0.f;
             bool ok = true;
-            for (int j = 0; j < n; ++j) {
+            for (int j = a; j < n; ++j) {
                 if (!wait_warp(&s_full[s], s_ph, sf)) { ok = false; break; }
                 s_ph ^= 1u;
                 ptx::tc_fence_after();
@@ -579,14 +619,20 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 ptx::tmem_ld32(tS + 96, &x[96]);
                 ptx::tmem_wait_ld();
                 mask_cols<0, 128>(x, kbase, lim);
+                if (WINDOW) mask_cols_below<0, 128>(x, kbase, first);
                 mx = fmaxf(row_max64<0>(x), row_max64<64>(x)) * sl2;
-                if (j == 0) {
+                if (j == a) {
                     m = mx;  // O is not written yet: the first P V overwrites it
                 } else if (mx - m > kLazyThreshold) {
+                    // (also taken when m is still -inf: the row's window had not started)
                     alpha = ptx::ex2(m - mx);
                     m = mx;
                     rescale = true;
                 }
+                // reference maximum for the exponentials: with a window, 0 while the row
+                // has seen no key, so that masked scores give exactly 0 instead of
+                // -inf - (-inf).  (Without one, every row sees a key in its first tile.)
+                const float mref = (WINDOW && m == -INFINITY) ? 0.f : m;
                 // Rare (lazy) rescale of the partial output, before any P V of this tile is
                 // issued (P V of the previous tile is complete: the commit that signalled
                 // this S tile covers it); warp-uniform because TMEM accesses are collective.
@@ -608,21 +654,21 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     // the first 64 keys of P are handed to the MMA warp while the second
                     // half is still being computed
                     rescale_o();
-                    sum = exp2_pack<64, 0, 0>(x, sl2, m);
+                    sum = exp2_pack<64, 0, 0>(x, sl2, mref);
                     ptx::tmem_st32(tS + 0, &x[0]);
                     ptx::tmem_wait_st();
                     ptx::tc_fence_before();
                     ptx::mbar_arrive(&p_half[s]);
-                    sum += exp2_pack<64, 64, 32>(x, sl2, m);
+                    sum += exp2_pack<64, 64, 32>(x, sl2, mref);
                     ptx::tmem_st32(tS + 32, &x[32]);
                 } else {
-                    sum = exp2_pack<64, 0, 0>(x, sl2, m) + exp2_pack<64, 64, 32>(x, sl2, m);
+                    sum = exp2_pack<64, 0, 0>(x, sl2, mref) + exp2_pack<64, 64, 32>(x, sl2, mref);
                     ptx::tmem_st32(tS + 0, &x[0]);
                     ptx::tmem_st32(tS + 32, &x[32]);
                     rescale_o();
                 }
                 ptx::tmem_wait_st();
-                const float p_top = ptx::ex2(mx - m);  // the tile's largest weight (0 if masked)
+                const float p_top = ptx::ex2(mx - mref);  // the tile's largest weight (0 if masked)
                 const float p_top_bf = __uint_as_float(ptx::pack_bf16x2(p_top, 0.f) << 16);
                 l = l * alpha + sum;
                 lo = lo * alpha + sum + (p_top_bf - p_top);

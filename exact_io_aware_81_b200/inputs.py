@@ -35,6 +35,7 @@ class Prefill:
     causal: bool
     scale: float
     out_dtype: torch.dtype
+    window: int = 0   # sliding window W (causal only); 0 = none
 
     @property
     def shape(self):
@@ -45,7 +46,7 @@ class Prefill:
     def pairs(self) -> int:
         """Number of (query row, key) pairs that the mask allows, summed over B and Hq."""
         B, Hq, Hkv, Nq, Nk, d = self.shape
-        return B * Hq * allowed_pairs(Nq, Nk, self.causal)
+        return B * Hq * allowed_pairs(Nq, Nk, self.causal, self.window)
 
     def flops(self) -> float:
         """Algorithmic flops: 2*d for q.k plus 2*d for p*v, per allowed pair."""
@@ -89,17 +90,24 @@ class Decode:
         return 4.0 * Hq * d * float(self.seqlens.to(torch.int64).sum().item())
 
 
-def allowed_pairs(Nq: int, Nk: int, causal: bool) -> int:
+def allowed_pairs(Nq: int, Nk: int, causal: bool, window: int = 0) -> int:
     """Pairs (i, j) with key j visible to query i.
 
     Causal masks use bottom-right alignment (row i sees keys 0 .. i + Nk - Nq), which
-    requires Nq <= Nk; every row then sees i + Nk - Nq + 1 keys.
+    requires Nq <= Nk; every row then sees c_i = i + Nk - Nq + 1 keys, or min(c_i, W)
+    with a sliding window of W keys.
     """
     if not causal:
         return Nq * Nk
     assert Nq <= Nk
     off = Nk - Nq
-    return Nq * (off + 1) + Nq * (Nq - 1) // 2
+    if window <= 0 or window >= Nk:
+        return Nq * (off + 1) + Nq * (Nq - 1) // 2
+    lo, hi = off + 1, Nk            # c_i runs over lo .. hi
+    top = min(hi, window)           # rows with c_i <= W see all c_i keys
+    full = (top - lo + 1) * (lo + top) // 2 if top >= lo else 0
+    capped = hi - max(lo, window + 1) + 1
+    return full + window * max(0, capped)
 
 
 def _randn(gen, shape, std=None):
@@ -114,7 +122,7 @@ def make_prefill(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, *, seed: i
                  out_dtype: torch.dtype = torch.bfloat16,
                  head_std_range: Optional[tuple] = None,
                  outlier_rows_frac: float = 0.0, outlier_factor: float = 3.0,
-                 name: str = "prefill") -> Prefill:
+                 window: int = 0, name: str = "prefill") -> Prefill:
     """Draw a seeded prefill problem.
 
     head_std_range=(lo, hi): each Q head and each K and V head gets its own standard
@@ -144,7 +152,7 @@ def make_prefill(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, *, seed: i
         scale = 1.0 / math.sqrt(d)
     return Prefill(name=name, q=q.to(torch.bfloat16), k=k.to(torch.bfloat16),
                    v=v.to(torch.bfloat16), causal=causal, scale=float(scale),
-                   out_dtype=out_dtype)
+                   out_dtype=out_dtype, window=int(window))
 
 
 def make_decode(B: int, Hq: int, Hkv: int, Nmax: int, d: int, *, seed: int,
@@ -173,6 +181,10 @@ WORKLOADS = {
     3: "gqa_causal_prefill_b4_hq32_hkv8_n8192_d128",
     4: "gqa_causal_prefill_b1_hq32_hkv8_n32768_d128_headstd",
     5: "gqa_decode_b32_hq32_hkv8_nmax8192_d128",
+    # sliding window and chunked prefill (youngju.dev sections 4 and 5), same head layout
+    6: "gqa_swa_prefill_b1_hq32_hkv8_n32768_w4096_d128",
+    7: "gqa_chunked_prefill_b1_hq32_hkv8_nq4096_nk32768_d128",
+    8: "gqa_swa_chunked_prefill_b4_hq32_hkv8_nq2048_nk16384_w4096_d128",
 }
 
 
@@ -193,6 +205,14 @@ def workload(k: int):
                             head_std_range=(0.5, 2.0), name=name)
     if k == 5:
         return make_decode(32, 32, 8, 8192, 128, seed=seed, len_range=(1024, 8192), name=name)
+    if k == 6:
+        return make_prefill(1, 32, 8, 32768, 32768, 128, seed=seed, causal=True, window=4096,
+                            name=name)
+    if k == 7:
+        return make_prefill(1, 32, 8, 4096, 32768, 128, seed=seed, causal=True, name=name)
+    if k == 8:
+        return make_prefill(4, 32, 8, 2048, 16384, 128, seed=seed, causal=True, window=4096,
+                            name=name)
     raise KeyError(k)
 
 

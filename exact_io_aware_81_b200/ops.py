@@ -33,6 +33,7 @@ _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "fa_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
@@ -103,12 +104,14 @@ def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale: Optional[float] = None, out_dtype: torch.dtype = torch.bfloat16,
         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-        stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+        stream=None, window: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
     """Attention forward: q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d) bf16 -> (o, lse).
 
     scale defaults to 1/sqrt(d) (as flash_attn_func's softmax_scale=None does on the
     toolsku.com page).  causal uses bottom-right alignment (row i sees keys up to
-    i + Nk - Nq).  o has out_dtype (bf16 or fp32); lse is fp32 (B,Hq,Nq), natural log.
+    i + Nk - Nq).  window = W >= 1 (causal only) restricts row i to its W most recent
+    keys (fa_fwd_window); 0 means no window.  o has out_dtype (bf16 or fp32); lse is
+    fp32 (B,Hq,Nq), natural log.
     """
     _require(q, "q", torch.bfloat16, 4)
     _require(k, "k", torch.bfloat16, 4)
@@ -129,12 +132,31 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     else:
         _require(lse, "lse", torch.float32, 3)
-    rc = load().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                          lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
-                          FA_F32 if out_dtype == torch.float32 else FA_BF16,
-                          _stream_handle(stream))
+    odt = FA_F32 if out_dtype == torch.float32 else FA_BF16
+    if window:
+        if not causal:
+            raise ValueError("a sliding window needs causal=True")
+        rc = load().fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(window),
+                                  odt, _stream_handle(stream))
+    else:
+        rc = load().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                              lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+                              odt, _stream_handle(stream))
     _check(rc)
     return out, lse
+
+
+def fwd_window(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int,
+               scale: Optional[float] = None, out_dtype: torch.dtype = torch.bfloat16,
+               out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+               stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Sliding-window causal attention (fa_fwd_window): row i sees keys j with
+    i + Nk - Nq - window < j <= i + Nk - Nq.  Arguments as fwd."""
+    if int(window) < 1:
+        raise ValueError("window must be >= 1")
+    return fwd(q, k, v, causal=True, scale=scale, out_dtype=out_dtype, out=out, lse=lse,
+               stream=stream, window=int(window))
 
 
 def decode_workspace_size(B: int, Hq: int, Nmax: int, d: int) -> int:

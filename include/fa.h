@@ -74,6 +74,21 @@ FA_API int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float
               int o_dtype, void *stream);
 
 /*
+ * Sliding-window causal attention (youngju.dev "attention variants", section 4: every
+ * token attends only to the W most recent tokens, itself included, so the cost falls
+ * from N^2 to N x W; with W = 3, query 5 sees keys 3, 4 and 5).  With the bottom-right
+ * alignment of fa_fwd, row i sees keys j with i + (Nk - Nq) - W < j <= i + (Nk - Nq);
+ * Nq < Nk is chunked prefill (youngju.dev section 5): the Nq new rows are the last Nq
+ * positions of a sequence whose first Nk - Nq keys are already cached.
+ *   window: W >= 1 (FA_ERR_INVALID otherwise); W >= Nk gives plain causal attention.
+ *   Key tiles that lie wholly outside every row's window are neither loaded nor
+ *   multiplied.  Other arguments, layouts, ownership and errors as fa_fwd_ex.
+ */
+FA_API int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse,
+                  int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
+                  int o_dtype, void *stream);
+
+/*
  * Bytes of device workspace fa_decode needs for these sizes (fp32 partial outputs and
  * partial log-sum-exps of the split-KV chunks).  0 if the sizes are invalid.
  */

@@ -115,3 +115,33 @@ def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.fwd(q, q, q)
+
+
+def _fwd_window(lib, window, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=4, Hkv=2, Nq=8, Nk=8, d=64,
+             scale=0.125, dt=0)
+    a.update(kw)
+    return lib.fa_fwd_window(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                             a["Nq"], a["Nk"], a["d"], a["scale"], window, a["dt"], None)
+
+
+@pytest.mark.parametrize("window,kw", [
+    (0, {}),                       # a window holds at least the row's own key
+    (-3, {}),
+    (4, dict(Nq=9, Nk=8)),         # causal (hence windowed) attention needs Nq <= Nk
+    (4, dict(d=96)),
+])
+def test_fwd_window_rejects(lib, window, kw):
+    rc = _fwd_window(lib, window, **kw)
+    assert rc in (ops.FA_ERR_INVALID, ops.FA_ERR_UNSUPPORTED) and rc != ops.FA_OK
+    if window <= 0 or kw.get("Nq", 0) > kw.get("Nk", 10 ** 9):
+        assert rc == ops.FA_ERR_INVALID
+
+
+def test_binding_window_needs_causal(lib):
+    import torch
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.fwd(q, q, q, causal=False, window=4)
+    with pytest.raises(ValueError):
+        ops.fwd_window(q, q, q, window=0)
