@@ -421,10 +421,11 @@ def run_ours(args, rank, world, local):
 
 
 def run_extra(args, dev, peaks):
-    """Per-workload kernel times for the other prefill workloads (not part of the step)."""
+    """Per-workload kernel times for the other prefill workloads (not part of the step):
+    the other causal shapes, sliding window (6, 8) and chunked prefill (7, 8)."""
     from exact_io_aware_81_b200 import ops
     res = {}
-    for kid in (1, 3, 4):
+    for kid in (1, 3, 4, 6, 7, 8):
         w = inputs.workload(kid)
         B, Hq, Hkv, Nq, Nk, d = w.shape
         q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
@@ -432,11 +433,13 @@ def run_extra(args, dev, peaks):
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
         n = 3 if kid != 1 else 20
         for _ in range(3):
-            ops.fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse)
+            ops.fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse,
+                    window=w.window)
         e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         e[0].record()
         for _ in range(n):
-            ops.fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse)
+            ops.fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse,
+                    window=w.window)
         e[1].record()
         torch.cuda.synchronize(dev)
         ms = e[0].elapsed_time(e[1]) / n

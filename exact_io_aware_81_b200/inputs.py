@@ -90,6 +90,41 @@ class Decode:
         return 4.0 * Hq * d * float(self.seqlens.to(torch.int64).sum().item())
 
 
+@dataclasses.dataclass
+class PagedDecode:
+    """One decode step over a paged cache: q (B,Hq,d); kpages/vpages
+    (num_pages,Hkv,page_size,d) bf16; block_table int32 (B,max_pages), -1 where unused;
+    seqlens int32[B].  Token t of sequence b is row t % page_size of physical page
+    block_table[b, t // page_size]."""
+    name: str
+    q: torch.Tensor
+    kpages: torch.Tensor
+    vpages: torch.Tensor
+    block_table: torch.Tensor
+    seqlens: torch.Tensor
+    scale: float
+
+    @property
+    def shape(self):
+        B, Hq, d = self.q.shape
+        num_pages, Hkv, page_size = self.kpages.shape[:3]
+        return B, Hq, Hkv, num_pages, page_size, self.block_table.shape[1], d
+
+    def cache_bytes(self) -> int:
+        B, Hq, Hkv, num_pages, page_size, max_pages, d = self.shape
+        return int(self.seqlens.to(torch.int64).sum().item()) * Hkv * d * 2 * 2
+
+    def io_bytes(self) -> int:
+        """Cache bytes, q read, bf16 o write, seqlens and the block-table entries used."""
+        B, Hq, Hkv, num_pages, page_size, max_pages, d = self.shape
+        pages_used = int(((self.seqlens.to(torch.int64) + page_size - 1) // page_size).sum().item())
+        return self.cache_bytes() + 2 * 2 * B * Hq * d + 4 * B + 4 * pages_used
+
+    def flops(self) -> float:
+        B, Hq, Hkv, num_pages, page_size, max_pages, d = self.shape
+        return 4.0 * Hq * d * float(self.seqlens.to(torch.int64).sum().item())
+
+
 def allowed_pairs(Nq: int, Nk: int, causal: bool, window: int = 0) -> int:
     """Pairs (i, j) with key j visible to query i.
 
@@ -173,7 +208,43 @@ def make_decode(B: int, Hq: int, Hkv: int, Nmax: int, d: int, *, seed: int,
                   vcache=vc.to(torch.bfloat16), seqlens=seqlens, scale=float(scale))
 
 
-# The five named workloads.  Sizes follow the pages' examples (H=32 and d_k=128 in the
+def make_paged_decode(B: int, Hq: int, Hkv: int, page_size: int, max_pages: int, d: int, *,
+                      seed: int, len_range: tuple, num_pages: Optional[int] = None,
+                      scale: Optional[float] = None, name: str = "paged_decode") -> PagedDecode:
+    """Draw a seeded decode step over a paged cache.
+
+    Draw order: seqlens (uniform on the inclusive ``len_range``) -> a random permutation
+    of the pool's pages, handed out in order to sequence 0's logical pages, then sequence
+    1's, ... (so a sequence's pages are scattered over the pool) -> q -> kpages -> vpages.
+    The pool holds ``num_pages`` pages (default: B * max_pages, room for every sequence at
+    full length); block-table entries past a sequence's last page are -1.
+    """
+    assert Hq % Hkv == 0
+    num_pages = num_pages or B * max_pages
+    gen = torch.Generator("cpu")
+    gen.manual_seed(seed)
+    lo, hi = len_range
+    assert 0 <= lo <= hi <= page_size * max_pages
+    seqlens = torch.randint(lo, hi + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+    need = ((seqlens.to(torch.int64) + page_size - 1) // page_size).tolist()
+    assert sum(need) <= num_pages, "pool too small"
+    perm = torch.randperm(num_pages, generator=gen).to(torch.int32)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    used = 0
+    for b in range(B):
+        table[b, :need[b]] = perm[used:used + need[b]]
+        used += need[b]
+    q = _randn(gen, (B, Hq, d))
+    kp = _randn(gen, (num_pages, Hkv, page_size, d))
+    vp = _randn(gen, (num_pages, Hkv, page_size, d))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    return PagedDecode(name=name, q=q.to(torch.bfloat16), kpages=kp.to(torch.bfloat16),
+                       vpages=vp.to(torch.bfloat16), block_table=table, seqlens=seqlens,
+                       scale=float(scale))
+
+
+# The named workloads.  1-5 follow the pages' examples (H=32 and d_k=128 in the
 # cost analysis, G=8 in the grouped-query section, contexts from 2K up to 32K).
 WORKLOADS = {
     1: "mha_fwd_b1_h2_n256_d64_noncausal_f32out",
@@ -185,6 +256,8 @@ WORKLOADS = {
     6: "gqa_swa_prefill_b1_hq32_hkv8_n32768_w4096_d128",
     7: "gqa_chunked_prefill_b1_hq32_hkv8_nq4096_nk32768_d128",
     8: "gqa_swa_chunked_prefill_b4_hq32_hkv8_nq2048_nk16384_w4096_d128",
+    # decode 5 over a paged cache of 64-token pages (youngju.dev section 5)
+    9: "gqa_paged_decode_b32_hq32_hkv8_page64_nmax8192_d128",
 }
 
 
@@ -213,6 +286,9 @@ def workload(k: int):
     if k == 8:
         return make_prefill(4, 32, 8, 2048, 16384, 128, seed=seed, causal=True, window=4096,
                             name=name)
+    if k == 9:
+        return make_paged_decode(32, 32, 8, 64, 8192 // 64, 128, seed=seed, len_range=(1024, 8192),
+                                 name=name)
     raise KeyError(k)
 
 

@@ -5,8 +5,8 @@ may import this package.  It shares no code with the CUDA path (``exact_io_aware
 and never imports it; the two meet only through the seeded inputs.
 
 Contents:
-  * ``attn_fwd`` / ``decode`` / ``probs``: the fp64 two-pass definition, in plain C with
-    OpenMP (``attn_oracle.c``), called through ctypes.
+  * ``attn_fwd`` / ``decode`` / ``decode_paged`` / ``probs``: the fp64 two-pass
+    definition, in plain C with OpenMP (``attn_oracle.c``), called through ctypes.
   * ``online.online_attention``: a restatement of the block-by-block online softmax
     (youngju.dev "attention variants", section 3), used only to check that the online
     and two-pass forms agree.
@@ -51,9 +51,11 @@ def declare(lib):
     lib.oracle_attn_probs.argtypes = [P, P, I, I, I, I, I, I, D, I, P]
     lib.oracle_attn_probs_window.argtypes = [P, P, I, I, I, I, I, I, D, I, I, P]
     lib.oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, D, P, P]
+    lib.oracle_decode_paged.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, P]
     lib.oracle_num_threads.argtypes = []
     for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_window, lib.oracle_attn_probs,
-              lib.oracle_attn_probs_window, lib.oracle_decode, lib.oracle_num_threads):
+              lib.oracle_attn_probs_window, lib.oracle_decode, lib.oracle_decode_paged,
+              lib.oracle_num_threads):
         f.restype = I
     return lib
 
@@ -143,4 +145,25 @@ def decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens:
                                float(scale), _ptr(o), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_decode rejected its arguments")
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def decode_paged(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor,
+                 block_table: torch.Tensor, seqlens: torch.Tensor, scale: float):
+    """fp64 decode over a paged cache: q (B,Hq,d); kpages/vpages (num_pages,Hkv,page_size,d);
+    block_table int32 (B,max_pages); token t of sequence b is row t % page_size of page
+    block_table[b, t // page_size]."""
+    B, Hq, d = q.shape
+    num_pages, Hkv, page_size = kpages.shape[0], kpages.shape[1], kpages.shape[2]
+    max_pages = block_table.shape[1]
+    qb, kb, vb = _bits(q), _bits(kpages), _bits(vpages)
+    bt = np.ascontiguousarray(block_table.detach().cpu().numpy().astype(np.int32))
+    sl = np.ascontiguousarray(seqlens.detach().cpu().numpy().astype(np.int32))
+    o = np.empty((B, Hq, d), dtype=np.float64)
+    lse = np.empty((B, Hq), dtype=np.float64)
+    rc = _load().oracle_decode_paged(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(bt), _ptr(sl), B, Hq, Hkv,
+                                     num_pages, page_size, max_pages, d, float(scale),
+                                     _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_decode_paged rejected its arguments")
     return torch.from_numpy(o), torch.from_numpy(lse)

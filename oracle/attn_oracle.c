@@ -245,6 +245,73 @@ int oracle_decode(const uint16_t *q, const uint16_t *kcache, const uint16_t *vca
     return err ? -1 : 0;
 }
 
+/*
+ * Decode over a paged KV cache (youngju.dev "attention variants", section 5: the cache is
+ * cut into fixed-size blocks managed like virtual-memory pages).  The page layout is this
+ * library's reading, the pages fix none:
+ *   kpages, vpages: (num_pages, Hkv, page_size, d) -- a page holds page_size consecutive
+ *                   tokens of one sequence, for every K/V head;
+ *   block_table:    int32 (B, max_pages): logical page t / page_size of sequence b is
+ *                   physical page block_table[b * max_pages + t / page_size], and token t
+ *                   is row t % page_size of it.
+ * Sequence b attends its first seqlens[b] tokens, exactly as oracle_decode does on a
+ * contiguous cache: each (b, K/V head) is first gathered into a contiguous buffer.
+ * Returns -1 on an argument error or a block-table entry outside [0, num_pages).
+ */
+int oracle_decode_paged(const uint16_t *q, const uint16_t *kpages, const uint16_t *vpages,
+                        const int32_t *block_table, const int32_t *seqlens,
+                        int B, int Hq, int Hkv, int num_pages, int page_size, int max_pages,
+                        int d, double scale, double *o, double *lse)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || num_pages <= 0 || page_size <= 0 || max_pages <= 0 ||
+        d <= 0)
+        return -1;
+    if (Hq % Hkv != 0) return -1;
+    const long cap = (long)page_size * max_pages;
+    for (int b = 0; b < B; ++b) {
+        if (seqlens[b] < 0 || seqlens[b] > cap) return -1;
+        for (long t = 0; t < ((long)seqlens[b] + page_size - 1) / page_size; ++t) {
+            int32_t pg = block_table[(long)b * max_pages + t];
+            if (pg < 0 || pg >= num_pages) return -1;
+        }
+    }
+    const long R = Hq / Hkv;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *qbuf = (double *)malloc(sizeof(double) * (size_t)d);
+        double *s = (double *)malloc(sizeof(double) * (size_t)cap);
+        uint16_t *kg = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)cap * d);
+        uint16_t *vg = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)cap * d);
+        if (!qbuf || !s || !kg || !vg) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bg = 0; bg < (long)B * Hkv; ++bg) {
+                long b = bg / Hkv, g = bg % Hkv;
+                long L = seqlens[b];
+                for (long t = 0; t < L; ++t) {
+                    long page = block_table[b * max_pages + t / page_size];
+                    long row = t % page_size;
+                    const long src = ((page * Hkv + g) * page_size + row) * d;
+                    memcpy(kg + t * d, kpages + src, sizeof(uint16_t) * (size_t)d);
+                    memcpy(vg + t * d, vpages + src, sizeof(uint16_t) * (size_t)d);
+                }
+                for (long h = g * R; h < (g + 1) * R; ++h) {
+                    long idx = b * Hq + h;
+                    attend_row(q + idx * d, kg, vg, L, d, scale, qbuf, s, o + idx * d, lse + idx);
+                }
+            }
+        }
+        free(qbuf);
+        free(s);
+        free(kg);
+        free(vg);
+    }
+    return err ? -1 : 0;
+}
+
 /* Number of OpenMP threads a parallel region would use (for reporting). */
 int oracle_num_threads(void)
 {

@@ -308,6 +308,62 @@ def pin_window_special_cases():
             assert abs(l1[0, h, i].item() - 0.7 * dot) < 1e-12
 
 
+def _scatter_to_pages(kc, seqlens, page_size, max_pages, num_pages, seed):
+    """Scatter a contiguous cache (B,Hkv,Nmax,d) into a page pool in a random page order;
+    returns (pool, block_table).  Plain indexing only."""
+    B, Hkv, Nmax, d = kc.shape
+    g = torch.Generator("cpu").manual_seed(seed)
+    perm = torch.randperm(num_pages, generator=g)
+    pool = torch.zeros((num_pages, Hkv, page_size, d), dtype=kc.dtype)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    used = 0
+    for b in range(B):
+        for t in range(-(-int(seqlens[b]) // page_size)):
+            pg = int(perm[used]); used += 1
+            table[b, t] = pg
+            rows = kc[b, :, t * page_size:(t + 1) * page_size]
+            pool[pg, :, :rows.shape[1]] = rows
+    return pool, table
+
+
+def pin_paged_decode_equals_contiguous():
+    """A cache scattered over pages in random order decodes exactly as the contiguous
+    cache, and as torch fp64 SDPA on the keys gathered back by plain indexing."""
+    B, Hq, Hkv, d = 4, 8, 2, 32
+    for page_size, max_pages in [(16, 20), (48, 7), (1, 300)]:
+        Nmax = page_size * max_pages
+        w = inputs.make_decode(B, Hq, Hkv, Nmax, d, seed=60 + page_size, len_range=(0, Nmax))
+        sl = torch.tensor([0, 1, Nmax, Nmax // 2 + 3], dtype=torch.int32)
+        num_pages = B * max_pages + 5
+        kp, table = _scatter_to_pages(w.kcache, sl, page_size, max_pages, num_pages, 70)
+        vp, table2 = _scatter_to_pages(w.vcache, sl, page_size, max_pages, num_pages, 70)
+        assert torch.equal(table, table2)
+        o, lse = oracle.decode_paged(w.q, kp, vp, table, sl, w.scale)
+        oc, lc = oracle.decode(w.q, w.kcache, w.vcache, sl, w.scale)
+        assert torch.equal(o, oc) and torch.equal(lse, lc), page_size
+        for b in range(1, B):
+            L = int(sl[b])
+            idx = torch.arange(L)
+            pages = table[b, idx // page_size].long()
+            kg = kp[pages, :, idx % page_size].permute(1, 0, 2).unsqueeze(0)
+            vg = vp[pages, :, idx % page_size].permute(1, 0, 2).unsqueeze(0)
+            ro, rl = _sdpa_ref(w.q[b:b + 1].unsqueeze(2), kg.contiguous(), vg.contiguous(), w.scale, False)
+            assert torch.allclose(o[b], ro[0, :, 0], atol=1e-12, rtol=0)
+            assert torch.allclose(lse[b], rl[0, :, 0], atol=1e-12, rtol=0)
+
+
+def pin_paged_generator_tables_are_valid():
+    """The seeded paged workloads: every used page is distinct and in range; unused -1."""
+    w = inputs.make_paged_decode(5, 4, 2, 16, 9, 16, seed=3, len_range=(0, 144))
+    B, Hq, Hkv, num_pages, ps, mp, d = w.shape
+    used = []
+    for b in range(B):
+        n = -(-int(w.seqlens[b]) // ps)
+        assert (w.block_table[b, n:] == -1).all()
+        used += w.block_table[b, :n].tolist()
+    assert len(set(used)) == len(used) and all(0 <= u < num_pages for u in used)
+
+
 PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]
 
 
@@ -331,6 +387,9 @@ MUTANTS = [
     ("last key dropped", "for (long j = 0; j < nkeys; ++j) {\n        double p", "for (long j = 0; j + 1 < nkeys; ++j) {\n        double p"),
     ("window off by one", "long first = i + (Nk - Nq) - window + 1;", "long first = i + (Nk - Nq) - window;"),
     ("window offset dropped", "long first = i + (Nk - Nq) - window + 1;", "long first = i - window + 1;"),
+    ("paged pool layout", "const long src = ((page * Hkv + g) * page_size + row) * d;",
+     "const long src = ((g * num_pages + page) * page_size + row) * d;"),
+    ("paged head map", "for (long h = g * R; h < (g + 1) * R; ++h)", "for (long h = g; h < Hq; h += Hkv)"),
 ]
 
 
