@@ -49,7 +49,7 @@ struct DeviceInfo {
     bool sm100 = false;
     int num_sms = 0;
     bool prefill_attr_set[2][2][2][2] = {};
-    bool decode_attr_set[2][4] = {{false, false, false, false}, {false, false, false, false}};
+    bool decode_attr_set[2][4][2] = {};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -243,16 +243,16 @@ size_t decode_ws_bytes(int B, int Hq, int Nmax, int d)
 }
 
 // Persistent split kernel: one CTA per SM (at most one per work item).
-template <int D, int RG>
+template <int D, int RG, bool PAGED>
 int launch_split(fa::DecodeParams p, DeviceInfo *info, cudaStream_t st)
 {
     using C = fa::decode::SplitCfg<D, RG>;
     static_assert(C::kSmemBytes * fa::decode::kCtasPerSm <= 227 * 1024, "decode CTAs per SM do not fit");
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
-        bool &set = info->decode_attr_set[D == 128][RG == 8 ? 3 : RG == 4 ? 2 : RG == 2 ? 1 : 0];
+        bool &set = info->decode_attr_set[D == 128][RG == 8 ? 3 : RG == 4 ? 2 : RG == 2 ? 1 : 0][PAGED];
         if (!set) {
-            cudaError_t e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, RG>,
+            cudaError_t e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, RG, PAGED>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
             if (e != cudaSuccess)
                 return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -263,18 +263,18 @@ int launch_split(fa::DecodeParams p, DeviceInfo *info, cudaStream_t st)
     p.n_items = p.S_max * p.B * p.n_hg;
     const int max_ctas = fa::decode::kCtasPerSm * info->num_sms;
     const int grid = p.n_items < max_ctas ? p.n_items : max_ctas;
-    fa::fa_decode_split_kernel<D, RG><<<grid, fa::decode::kThreads, C::kSmemBytes, st>>>(p);
+    fa::fa_decode_split_kernel<D, RG, PAGED><<<grid, fa::decode::kThreads, C::kSmemBytes, st>>>(p);
     return FA_OK;
 }
 
-template <int D>
+template <int D, bool PAGED = false>
 int launch_split_rg(const fa::DecodeParams &p, int rg, DeviceInfo *info, cudaStream_t st)
 {
     switch (rg) {
-    case 8: return launch_split<D, 8>(p, info, st);
-    case 4: return launch_split<D, 4>(p, info, st);
-    case 2: return launch_split<D, 2>(p, info, st);
-    default: return launch_split<D, 1>(p, info, st);
+    case 8: return launch_split<D, 8, PAGED>(p, info, st);
+    case 4: return launch_split<D, 4, PAGED>(p, info, st);
+    case 2: return launch_split<D, 2, PAGED>(p, info, st);
+    default: return launch_split<D, 1, PAGED>(p, info, st);
     }
 }
 
@@ -385,6 +385,76 @@ int fa_decode(const void *q, const void *kcache, const void *vcache, const int *
     return ok();
 }
 
+int fa_decode_paged(const void *q, const void *kpages, const void *vpages, const int *block_table,
+                    const int *seqlens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
+                    int page_size, int max_pages, int d, float scale, void *workspace,
+                    size_t workspace_bytes, void *stream)
+{
+    if (!q || !kpages || !vpages || !block_table || !seqlens || !o)
+        return fail(FA_ERR_INVALID, "null pointer argument");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || num_pages <= 0 || page_size <= 0 || max_pages <= 0 || d <= 0)
+        return fail(FA_ERR_INVALID,
+                    "sizes must be positive (B=%d Hq=%d Hkv=%d num_pages=%d page_size=%d max_pages=%d d=%d)",
+                    B, Hq, Hkv, num_pages, page_size, max_pages, d);
+    if (Hq % Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(FA_ERR_INVALID, "scale must be finite and > 0");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    if (page_size % 16 != 0) return fail(FA_ERR_UNSUPPORTED, "page_size %d is not a multiple of 16", page_size);
+    if (!aligned16(q) || !aligned16(kpages) || !aligned16(vpages) || !aligned16(o))
+        return fail(FA_ERR_UNSUPPORTED, "q, kpages, vpages and o must be 16-byte aligned");
+    const long long nmax = (long long)page_size * max_pages;
+    if (B > 65535 || nmax > 0x7fffffffLL || (long long)num_pages * Hkv > 0x7fffffffLL)
+        return fail(FA_ERR_UNSUPPORTED, "problem too large");
+    const int Nmax = (int)nmax;
+    const size_t need = decode_ws_bytes(B, Hq, Nmax, d);
+    if (!workspace || workspace_bytes < need)
+        return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned16(workspace)) return fail(FA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    int dev, rc;
+    DeviceInfo *info;
+    if ((rc = current_device(&dev, &info)) != FA_OK) return rc;
+
+    const int R = Hq / Hkv;
+    const int rg = (R % 8 == 0) ? 8 : (R % 4 == 0) ? 4 : (R % 2 == 0) ? 2 : 1;
+    if (Hq / rg > 65535) return fail(FA_ERR_UNSUPPORTED, "too many head groups");
+
+    fa::DecodeParams p;
+    memset(&p, 0, sizeof p);
+    // rows per copy: the largest power of two that divides page_size, at most 64
+    p.box_rows = page_size & -page_size;
+    if (p.box_rows > fa::decode::kSub) p.box_rows = fa::decode::kSub;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    if ((rc = encode_rows_map(&p.tm_k, kpages, d, page_size, (long long)num_pages * Hkv, p.box_rows)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, vpages, d, page_size, (long long)num_pages * Hkv, p.box_rows)) != FA_OK) return rc;
+    p.block_table = block_table;
+    p.page_size = page_size;
+    p.max_pages = max_pages;
+    p.num_pages = num_pages;
+    p.seqlens = seqlens;
+    p.S_max = (int)decode_splits(Nmax);
+    p.part_o = static_cast<float *>(workspace);
+    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                           align256((size_t)B * Hq * p.S_max * d * sizeof(float)));
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nmax = Nmax;
+    p.R = R;
+    p.scale_log2 = scale * 1.4426950408889634f;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    p.wait_limit_ns = g_wait_limit_ns;
+    rc = (d == 128) ? launch_split_rg<128, true>(p, rg, info, st) : launch_split_rg<64, true>(p, rg, info, st);
+    if (rc != FA_OK) return rc;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "paged decode split launch: %s", cudaGetErrorString(e));
+    e = (d == 128) ? launch_merge<128>(p, st) : launch_merge<64>(p, st);
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 // ------------------------------------------------------------ allocation-free decode
 //
 // For callers that cannot allocate device memory (see fa_decode_noalloc in fa.h): the
@@ -489,6 +559,8 @@ int fa_get_error(void *stream)
     }
     if (word & fa::kErrTimeout) return fail(FA_ERR_TIMEOUT, "a kernel pipeline wait exceeded its time limit");
     if (word & fa::kErrSeqlenRange) return fail(FA_ERR_DEVICE_ARG, "seqlens held a value outside [0, Nmax]");
+    if (word & fa::kErrPageRange)
+        return fail(FA_ERR_DEVICE_ARG, "the block table held a page outside [0, num_pages)");
     return ok();
 }
 

@@ -11,6 +11,7 @@ namespace fa {
 enum : unsigned int {
     kErrTimeout = 1u,      // a pipeline wait exceeded its limit
     kErrSeqlenRange = 2u,  // a decode length was outside [0, Nmax] and was clamped
+    kErrPageRange = 4u,    // a block-table entry was outside [0, num_pages); its keys read as 0
 };
 
 // One word per process, in the library's own device memory.

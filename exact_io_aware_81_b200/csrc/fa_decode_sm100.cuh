@@ -18,6 +18,13 @@
 //     w_s = 2^(lse_s - M), o = sum_s w_s o_s / sum_s w_s, lse = M + log2 sum_s w_s.
 // The merge is the same rescaling the online softmax applies between key blocks
 // (youngju.dev section 3), applied across chunks.
+//
+// Paged caches (youngju.dev section 5: the cache cut into fixed-size blocks managed like
+// virtual-memory pages) change only the producer's addressing: the tensor maps span the
+// page pool (num_pages * Hkv planes of page_size rows), the producer warp looks up the
+// physical pages of an item's keys in the block table (one entry per lane) and copies
+// boxes of box_rows rows, a power of two that divides page_size, so no box straddles two
+// pages; the consumers and the merge are unchanged.
 #pragma once
 
 #include <cstdint>
@@ -29,8 +36,9 @@
 namespace fa {
 
 struct DecodeParams {
-    CUtensorMap tm_k;         // kcache as (D, Nmax, B*Hkv) bf16, box (64, 64, 1), 128B swizzle
-    CUtensorMap tm_v;         // vcache, same shape
+    CUtensorMap tm_k;         // kcache as (D, Nmax, B*Hkv) bf16, box (64, 64, 1), 128B swizzle;
+                              // paged: kpages as (D, page_size, num_pages*Hkv), box (64, box_rows, 1)
+    CUtensorMap tm_v;         // vcache / vpages, same shape
     const __nv_bfloat16 *q;   // (B, Hq, D)
     const int *seqlens;       // (B)
     float *part_o;            // (B, Hq, S_max, D)  normalised partial outputs
@@ -42,6 +50,10 @@ struct DecodeParams {
     int n_items;   // S_max * B * n_hg candidate work items (chunk-major order)
     float scale_log2;
     unsigned long long wait_limit_ns;
+    // paged cache only (Nmax = page_size * max_pages)
+    const int *block_table;   // (B, max_pages) physical page of each logical page
+    int page_size, max_pages, num_pages;
+    int box_rows;             // rows per copy: a power of two <= 64 that divides page_size
 };
 
 namespace decode {
@@ -105,7 +117,7 @@ __device__ __forceinline__ bool decode_item(const DecodeParams &p, int it, int &
 // (rows RG .. 15 are zero): S = Q K^T per 8-key column tile, O += P V per 8-column tile,
 // both with fp32 accumulation; K and V fragments come from the swizzled stages through
 // ldmatrix (transposed for V).
-template <int D, int RG>
+template <int D, int RG, bool PAGED>
 __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
     fa_decode_split_kernel(const __grid_constant__ DecodeParams p)
 {
@@ -159,14 +171,48 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
         for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
             int b, hg, start, n;
             if (!decode_item(p, it, b, hg, start, n)) continue;
-            const int plane = b * p.Hkv + hg * RG / p.R;
+            const int g = hg * RG / p.R;
+            const int plane = b * p.Hkv + g;
+            // paged: lane i holds the physical page of the item's i-th logical page (an
+            // item of kChunk keys spans at most kChunk / 16 + 1 <= 32 pages); an entry
+            // outside the pool is reported and replaced by one past the pool's end, whose
+            // copies read zeros
+            int first_lp = 0, my_page = 0;
+            if (PAGED) {
+                first_lp = start / p.page_size;
+                const int lp = first_lp + lane;
+                if (lp <= (start + n - 1) / p.page_size) {
+                    my_page = p.block_table[(size_t)b * p.max_pages + lp];
+                    if (my_page < 0 || my_page >= p.num_pages) {
+                        raise_error(kErrPageRange);
+                        my_page = p.num_pages;
+                    }
+                }
+            }
             for (int pass = 0; pass < 2 && ok; ++pass) {
                 const CUtensorMap *map = pass ? &p.tm_v : &p.tm_k;
                 for (int t = 0; t * kSub < n; ++t) {
                     const uint32_t st = ring % C::kStages;
                     const uint32_t ph = (ring / C::kStages) & 1u;
                     if (!wait_warp(&empty[st], ph ^ 1u, sf)) { ok = false; break; }
-                    if (leader) {
+                    if (PAGED) {
+                        // only the boxes that hold keys of the sequence are copied (rows past
+                        // it are masked or cleared by the consumers)
+                        const int nbox = (min(kSub, n - t * kSub) + p.box_rows - 1) / p.box_rows;
+                        if (leader) ptx::mbar_arrive_expect_tx(&full[st], nbox * p.box_rows * 128 * (D / 64));
+                        for (int i = 0; i < nbox; ++i) {
+                            const int key = start + t * kSub + i * p.box_rows;
+                            const int lp = key / p.page_size;
+                            const int page = __shfl_sync(0xffffffffu, my_page, lp - first_lp);
+                            if (leader) {
+#pragma unroll
+                                for (int c = 0; c < D / 64; ++c)
+                                    ptx::tma_load_3d(smem + st * C::kStageBytes + c * kBoxBytes + i * p.box_rows * 128,
+                                                     map, &full[st], 64 * c, key - lp * p.page_size,
+                                                     page * p.Hkv + g);
+                            }
+                        }
+                    } else if (leader) {
                         ptx::mbar_arrive_expect_tx(&full[st], C::kStageBytes);
 #pragma unroll
                         for (int c = 0; c < D / 64; ++c)

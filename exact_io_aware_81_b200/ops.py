@@ -37,6 +37,7 @@ SIGNATURES = {
     "fa_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_get_error": (_I, [_P]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "fa_fwd_selftest_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
@@ -199,6 +200,50 @@ def decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens:
                           out.data_ptr(), lse.data_ptr() if lse is not None else None,
                           B, Hq, Hkv, Nmax, d, float(scale), workspace.data_ptr(),
                           workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def decode_paged(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor,
+                 block_table: torch.Tensor, seqlens: torch.Tensor, scale: Optional[float] = None,
+                 workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
+    """Decode over a paged cache (fa_decode_paged): q (B,Hq,d); kpages/vpages
+    (num_pages,Hkv,page_size,d) bf16; block_table int32 (B,max_pages) and seqlens int32[B]
+    on the device.  Token t of sequence b is row t % page_size of page
+    block_table[b, t // page_size].  Returns (o, lse) as decode does."""
+    _require(q, "q", torch.bfloat16, 3)
+    _require(kpages, "kpages", torch.bfloat16, 4)
+    _require(vpages, "vpages", torch.bfloat16, 4)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, d = q.shape
+    num_pages, Hkv, page_size, dk = kpages.shape
+    max_pages = block_table.shape[1]
+    if (dk != d or tuple(vpages.shape) != tuple(kpages.shape) or seqlens.shape[0] != B
+            or block_table.shape[0] != B):
+        raise ValueError("shape mismatch between q, kpages, vpages, block_table and seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = decode_workspace_size(B, Hq, page_size * max_pages, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    elif not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    else:
+        _require(out, "out", torch.bfloat16, 3)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _require(lse, "lse", torch.float32, 2)
+    rc = load().fa_decode_paged(q.data_ptr(), kpages.data_ptr(), vpages.data_ptr(),
+                                block_table.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
+                                lse.data_ptr() if lse is not None else None, B, Hq, Hkv,
+                                num_pages, page_size, max_pages, d, float(scale),
+                                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                _stream_handle(stream))
     _check(rc)
     return out, lse
 

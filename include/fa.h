@@ -49,7 +49,8 @@ typedef enum {
     FA_ERR_WORKSPACE = 3,    /* decode workspace null or smaller than required */
     FA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed; see fa_last_error_message */
     FA_ERR_TIMEOUT = 5,      /* a kernel pipeline wait exceeded its time limit (fa_get_error) */
-    FA_ERR_DEVICE_ARG = 6    /* the device found seqlens[b] outside [0, Nmax] and clamped it */
+    FA_ERR_DEVICE_ARG = 6    /* the device found seqlens[b] outside [0, Nmax] and clamped it,
+                                or a block-table entry outside the page pool */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
@@ -112,6 +113,31 @@ FA_API size_t fa_decode_workspace_size(int B, int Hq, int Nmax, int d);
 FA_API int fa_decode(const void *q, const void *kcache, const void *vcache, const int *seqlens,
               void *o, float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale,
               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Decode step over a paged KV cache (youngju.dev "attention variants", section 5: the
+ * cache is cut into fixed-size blocks managed like virtual-memory pages, which removes
+ * fragmentation).  The page layout is this library's choice:
+ *   kpages, vpages  (num_pages, Hkv, page_size, d) bf16: a page holds page_size
+ *                   consecutive tokens of one sequence for every K/V head;
+ *   block_table     int32 (B, max_pages) in device memory: token t of sequence b is row
+ *                   t % page_size of page block_table[b * max_pages + t / page_size].
+ *                   Only the entries of pages 0 .. ceil(seqlens[b] / page_size) - 1 are
+ *                   read; each must lie in [0, num_pages).  An entry outside it is
+ *                   reported by fa_get_error as FA_ERR_DEVICE_ARG, and the keys of that
+ *                   page read as zeros (no memory outside the pool is touched).
+ *   seqlens         int32[B], each in [0, page_size * max_pages].
+ *   page_size       a multiple of 16 (FA_ERR_UNSUPPORTED otherwise).
+ *   workspace       at least fa_decode_workspace_size(B, Hq, page_size * max_pages, d)
+ *                   bytes, as for fa_decode.
+ * q, o, lse, scale, stream and the result are exactly those of fa_decode on the cache the
+ * pages spell out.
+ */
+FA_API int fa_decode_paged(const void *q, const void *kpages, const void *vpages,
+                    const int *block_table, const int *seqlens, void *o, float *lse,
+                    int B, int Hq, int Hkv, int num_pages, int page_size, int max_pages,
+                    int d, float scale, void *workspace, size_t workspace_bytes,
+                    void *stream);
 
 /*
  * Decode step that allocates nothing and takes no workspace (no counterpart on the

@@ -145,3 +145,33 @@ def test_binding_window_needs_causal(lib):
         ops.fwd(q, q, q, causal=False, window=4)
     with pytest.raises(ValueError):
         ops.fwd_window(q, q, q, window=0)
+
+
+def _paged(lib, **kw):
+    a = dict(q=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=None, B=2, Hq=8, Hkv=2,
+             num_pages=10, ps=64, mp=5, d=128, scale=0.1, ws=FAKE, wsb=None)
+    a.update(kw)
+    if a["wsb"] is None:
+        a["wsb"] = lib.fa_decode_workspace_size(a["B"], a["Hq"], a["ps"] * a["mp"], a["d"])
+    return lib.fa_decode_paged(a["q"], a["kp"], a["vp"], a["bt"], a["sl"], a["o"], a["lse"],
+                               a["B"], a["Hq"], a["Hkv"], a["num_pages"], a["ps"], a["mp"], a["d"],
+                               a["scale"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(bt=None), ops.FA_ERR_INVALID),
+    (dict(kp=None), ops.FA_ERR_INVALID),
+    (dict(num_pages=0), ops.FA_ERR_INVALID),
+    (dict(ps=0), ops.FA_ERR_INVALID),
+    (dict(mp=-1), ops.FA_ERR_INVALID),
+    (dict(Hq=8, Hkv=3), ops.FA_ERR_INVALID),
+    (dict(scale=float("nan")), ops.FA_ERR_INVALID),
+    (dict(ps=40), ops.FA_ERR_UNSUPPORTED),           # pages are multiples of 16 rows
+    (dict(ps=8), ops.FA_ERR_UNSUPPORTED),
+    (dict(d=96), ops.FA_ERR_UNSUPPORTED),
+    (dict(vp=FAKE + 8), ops.FA_ERR_UNSUPPORTED),
+    (dict(ws=None), ops.FA_ERR_WORKSPACE),
+    (dict(wsb=256), ops.FA_ERR_WORKSPACE),
+])
+def test_decode_paged_rejects(lib, kw, status):
+    assert _paged(lib, **kw) == status
