@@ -125,6 +125,86 @@ class PagedDecode:
         return 4.0 * Hq * d * float(self.seqlens.to(torch.int64).sum().item())
 
 
+@dataclasses.dataclass
+class Fp8Decode:
+    """One decode step over an FP8 E4M3 cache: q (B,Hq,d) bf16; kcache/vcache uint8
+    (B,Hkv,Nmax,d) holding E4M3 bytes; k_scale/v_scale float32 (Hkv,): key j of head g is
+    k_scale[g] * e4m3(kcache[b,g,j,:]) (likewise V); seqlens int32[B]."""
+    name: str
+    q: torch.Tensor
+    kcache: torch.Tensor
+    vcache: torch.Tensor
+    k_scale: torch.Tensor
+    v_scale: torch.Tensor
+    seqlens: torch.Tensor
+    scale: float
+
+    @property
+    def shape(self):
+        B, Hq, d = self.q.shape
+        Hkv, Nmax = self.kcache.shape[1], self.kcache.shape[2]
+        return B, Hq, Hkv, Nmax, d
+
+    def cache_bytes(self) -> int:
+        """K and V bytes the step must read: 2 tensors * Hkv * d * 1 B per cached token."""
+        B, Hq, Hkv, Nmax, d = self.shape
+        return int(self.seqlens.to(torch.int64).sum().item()) * Hkv * d * 2
+
+    def io_bytes(self) -> int:
+        B, Hq, Hkv, Nmax, d = self.shape
+        return self.cache_bytes() + 2 * 2 * B * Hq * d + 4 * B + 2 * 4 * Hkv
+
+    def flops(self) -> float:
+        B, Hq, Hkv, Nmax, d = self.shape
+        return 4.0 * Hq * d * float(self.seqlens.to(torch.int64).sum().item())
+
+
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x: torch.Tensor, head_dim: int = 1):
+    """Per-head FP8 E4M3 encoding of an fp32 tensor: scale[g] = max|x[:, g]| / 448 and
+    bytes = e4m3(x / scale) (torch's round-to-nearest-even cast, clamped to +-448).
+    Returns (uint8 bytes, float32 scales).  Used only to prepare cache contents."""
+    xt = x.transpose(0, head_dim)
+    amax = xt.reshape(xt.shape[0], -1).abs().amax(dim=1)
+    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax)).to(torch.float32)
+    shape = [1] * x.dim()
+    shape[head_dim] = -1
+    y = (x / scale.view(shape)).clamp(-E4M3_MAX, E4M3_MAX)
+    return y.to(torch.float8_e4m3fn).view(torch.uint8), scale
+
+
+def make_fp8_decode(B: int, Hq: int, Hkv: int, Nmax: int, d: int, *, seed: int,
+                    len_range: tuple, head_std_range: Optional[tuple] = (0.5, 2.0),
+                    scale: Optional[float] = None, name: str = "fp8_decode") -> Fp8Decode:
+    """Draw a seeded decode step over an FP8 cache.
+
+    Draw order: seqlens -> per-K/V-head standard deviations (uniform in head_std_range,
+    so every head gets its own scale) -> q -> K -> V, all fp32; K and V are then encoded
+    per head with quantize_e4m3.
+    """
+    assert Hq % Hkv == 0
+    gen = torch.Generator("cpu")
+    gen.manual_seed(seed)
+    lo, hi = len_range
+    seqlens = torch.randint(lo, hi + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+    k_std = v_std = None
+    if head_std_range is not None:
+        a, b_ = head_std_range
+        k_std = (a + (b_ - a) * torch.rand((Hkv,), generator=gen)).view(1, Hkv, 1, 1)
+        v_std = (a + (b_ - a) * torch.rand((Hkv,), generator=gen)).view(1, Hkv, 1, 1)
+    q = _randn(gen, (B, Hq, d))
+    kc = _randn(gen, (B, Hkv, Nmax, d), k_std)
+    vc = _randn(gen, (B, Hkv, Nmax, d), v_std)
+    kq, ks = quantize_e4m3(kc)
+    vq, vs = quantize_e4m3(vc)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    return Fp8Decode(name=name, q=q.to(torch.bfloat16), kcache=kq, vcache=vq, k_scale=ks,
+                     v_scale=vs, seqlens=seqlens, scale=float(scale))
+
+
 def allowed_pairs(Nq: int, Nk: int, causal: bool, window: int = 0) -> int:
     """Pairs (i, j) with key j visible to query i.
 
@@ -258,6 +338,8 @@ WORKLOADS = {
     8: "gqa_swa_chunked_prefill_b4_hq32_hkv8_nq2048_nk16384_w4096_d128",
     # decode 5 over a paged cache of 64-token pages (youngju.dev section 5)
     9: "gqa_paged_decode_b32_hq32_hkv8_page64_nmax8192_d128",
+    # decode 5 over an FP8 (E4M3) cache with per-head scales (youngju.dev sections 5, 7)
+    10: "gqa_fp8kv_decode_b32_hq32_hkv8_nmax8192_d128",
 }
 
 
@@ -289,6 +371,8 @@ def workload(k: int):
     if k == 9:
         return make_paged_decode(32, 32, 8, 64, 8192 // 64, 128, seed=seed, len_range=(1024, 8192),
                                  name=name)
+    if k == 10:
+        return make_fp8_decode(32, 32, 8, 8192, 128, seed=seed, len_range=(1024, 8192), name=name)
     raise KeyError(k)
 
 

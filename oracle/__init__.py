@@ -5,8 +5,9 @@ may import this package.  It shares no code with the CUDA path (``exact_io_aware
 and never imports it; the two meet only through the seeded inputs.
 
 Contents:
-  * ``attn_fwd`` / ``decode`` / ``decode_paged`` / ``probs``: the fp64 two-pass
-    definition, in plain C with OpenMP (``attn_oracle.c``), called through ctypes.
+  * ``attn_fwd`` / ``decode`` / ``decode_paged`` / ``decode_fp8`` / ``probs``: the fp64
+    two-pass definition, in plain C with OpenMP (``attn_oracle.c``), called through
+    ctypes; ``e4m3_to_double`` decodes one FP8 E4M3 byte.
   * ``online.online_attention``: a restatement of the block-by-block online softmax
     (youngju.dev "attention variants", section 3), used only to check that the online
     and two-pass forms agree.
@@ -52,10 +53,13 @@ def declare(lib):
     lib.oracle_attn_probs_window.argtypes = [P, P, I, I, I, I, I, I, D, I, I, P]
     lib.oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, D, P, P]
     lib.oracle_decode_paged.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, P]
+    lib.oracle_decode_fp8.argtypes = [P, P, P, P, P, P, I, I, I, I, I, D, P, P]
+    lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_to_double.restype = D
     lib.oracle_num_threads.argtypes = []
     for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_window, lib.oracle_attn_probs,
               lib.oracle_attn_probs_window, lib.oracle_decode, lib.oracle_decode_paged,
-              lib.oracle_num_threads):
+              lib.oracle_decode_fp8, lib.oracle_num_threads):
         f.restype = I
     return lib
 
@@ -166,4 +170,31 @@ def decode_paged(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor,
                                      _ptr(o), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_decode_paged rejected its arguments")
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def e4m3_to_double(x: int) -> float:
+    """Value of one FP8 E4M3 byte (OCP "e4m3fn": bias 7, no infinities, S.1111.111 = NaN)."""
+    return float(_load().oracle_e4m3_to_double(int(x) & 0xFF))
+
+
+def decode_fp8(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor,
+               k_scale: torch.Tensor, v_scale: torch.Tensor, seqlens: torch.Tensor, scale: float):
+    """fp64 decode over an FP8 E4M3 cache: kcache/vcache uint8 (B,Hkv,Nmax,d) holding E4M3
+    bytes; key j of head g is k_scale[g] * e4m3(byte) (likewise V with v_scale)."""
+    B, Hq, d = q.shape
+    Hkv, Nmax = kcache.shape[1], kcache.shape[2]
+    assert kcache.dtype == torch.uint8 and vcache.dtype == torch.uint8
+    qb = _bits(q)
+    kb = np.ascontiguousarray(kcache.detach().cpu().numpy())
+    vb = np.ascontiguousarray(vcache.detach().cpu().numpy())
+    ks = np.ascontiguousarray(k_scale.detach().cpu().numpy().astype(np.float32))
+    vs = np.ascontiguousarray(v_scale.detach().cpu().numpy().astype(np.float32))
+    sl = np.ascontiguousarray(seqlens.detach().cpu().numpy().astype(np.int32))
+    o = np.empty((B, Hq, d), dtype=np.float64)
+    lse = np.empty((B, Hq), dtype=np.float64)
+    rc = _load().oracle_decode_fp8(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(ks), _ptr(vs), _ptr(sl),
+                                   B, Hq, Hkv, Nmax, d, float(scale), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_decode_fp8 rejected its arguments")
     return torch.from_numpy(o), torch.from_numpy(lse)

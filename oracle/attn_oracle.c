@@ -312,6 +312,102 @@ int oracle_decode_paged(const uint16_t *q, const uint16_t *kpages, const uint16_
     return err ? -1 : 0;
 }
 
+/*
+ * OCP FP8 E4M3 (the "e4m3fn" variant): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+ * bits.  Exponent field 0 holds the subnormals (m / 8) * 2^-6; exponent 15 with mantissa 7
+ * is NaN; there are no infinities, so the largest magnitude is 1.75 * 2^8 = 448.
+ */
+double oracle_e4m3_to_double(uint8_t x)
+{
+    int e = (x >> 3) & 15, m = x & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (x & 0x80) ? -v : v;
+}
+
+/* One query row against nkeys dequantized key/value rows (doubles, row-major nkeys x d):
+ * the same two passes as attend_row. */
+static void attend_row_dq(const uint16_t *qrow, const double *kd, const double *vd, long nkeys,
+                          long d, double scale, double *qbuf, double *s, double *orow,
+                          double *lse)
+{
+    for (long t = 0; t < d; ++t) qbuf[t] = bf16_bits_to_double(qrow[t]);
+    for (long t = 0; t < d; ++t) orow[t] = 0.0;
+    if (nkeys <= 0) { *lse = -INFINITY; return; }
+    for (long j = 0; j < nkeys; ++j) {
+        double acc = 0.0;
+        for (long t = 0; t < d; ++t) acc += qbuf[t] * kd[j * d + t];
+        s[j] = scale * acc;
+    }
+    double mx = s[0];
+    for (long j = 1; j < nkeys; ++j) if (s[j] > mx) mx = s[j];
+    double sum = 0.0;
+    for (long j = 0; j < nkeys; ++j) sum += exp(s[j] - mx);
+    for (long j = 0; j < nkeys; ++j) {
+        double w = exp(s[j] - mx) / sum;
+        for (long t = 0; t < d; ++t) orow[t] += w * vd[j * d + t];
+    }
+    *lse = mx + log(sum);
+}
+
+/*
+ * Decode over an FP8 (E4M3) KV cache.  The pages name FP8 KV caches (youngju.dev
+ * "attention variants", sections 5 and 7) but fix no scale convention; this library's
+ * reading is one dequantization scale per K/V head for K and one for V:
+ *   key   j of head g = k_scale[g] * e4m3(kcache[b, g, j, :])
+ *   value j of head g = v_scale[g] * e4m3(vcache[b, g, j, :])
+ * (a single per-tensor scale is the case of equal entries).  Everything else is
+ * oracle_decode: q bf16 (B,Hq,d), caches (B,Hkv,Nmax,d) bytes, seqlens in [0, Nmax].
+ */
+int oracle_decode_fp8(const uint16_t *q, const uint8_t *kcache, const uint8_t *vcache,
+                      const float *k_scale, const float *v_scale, const int32_t *seqlens,
+                      int B, int Hq, int Hkv, int Nmax, int d, double scale, double *o,
+                      double *lse)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nmax <= 0 || d <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > Nmax) return -1;
+    const long R = Hq / Hkv;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *qbuf = (double *)malloc(sizeof(double) * (size_t)d);
+        double *s = (double *)malloc(sizeof(double) * (size_t)Nmax);
+        double *kd = (double *)malloc(sizeof(double) * (size_t)Nmax * d);
+        double *vd = (double *)malloc(sizeof(double) * (size_t)Nmax * d);
+        if (!qbuf || !s || !kd || !vd) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bg = 0; bg < (long)B * Hkv; ++bg) {
+                long b = bg / Hkv, g = bg % Hkv;
+                long L = seqlens[b];
+                const uint8_t *kh = kcache + bg * (long)Nmax * d;
+                const uint8_t *vh = vcache + bg * (long)Nmax * d;
+                for (long e = 0; e < L * d; ++e) {
+                    kd[e] = (double)k_scale[g] * oracle_e4m3_to_double(kh[e]);
+                    vd[e] = (double)v_scale[g] * oracle_e4m3_to_double(vh[e]);
+                }
+                for (long h = g * R; h < (g + 1) * R; ++h) {
+                    long idx = b * Hq + h;
+                    attend_row_dq(q + idx * d, kd, vd, L, d, scale, qbuf, s, o + idx * d, lse + idx);
+                }
+            }
+        }
+        free(qbuf);
+        free(s);
+        free(kd);
+        free(vd);
+    }
+    return err ? -1 : 0;
+}
+
 /* Number of OpenMP threads a parallel region would use (for reporting). */
 int oracle_num_threads(void)
 {

@@ -364,6 +364,58 @@ def pin_paged_generator_tables_are_valid():
     assert len(set(used)) == len(used) and all(0 <= u < num_pages for u in used)
 
 
+def pin_e4m3_decoding():
+    """E4M3 bytes by hand from the format (bias 7, subnormals m/8 * 2^-6, S.1111.111 NaN,
+    max 448), and all 256 against torch's float8_e4m3fn conversion."""
+    by_hand = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0,
+               0x3F: 1.875, 0x40: 2.0, 0x41: 2.25, 0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0,
+               0x30: 0.5, 0x58: 16.0}
+    for x, want in by_hand.items():
+        assert oracle.e4m3_to_double(x) == want, hex(x)
+    assert math.isnan(oracle.e4m3_to_double(0x7F)) and math.isnan(oracle.e4m3_to_double(0xFF))
+    assert math.copysign(1.0, oracle.e4m3_to_double(0x80)) == -1.0
+    lib = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double()
+    for x in range(256):
+        a, b = oracle.e4m3_to_double(x), lib[x].item()
+        assert (math.isnan(a) and math.isnan(b)) or a == b, hex(x)
+
+
+def _dequant(bytes_u8, scales):
+    return bytes_u8.view(torch.float8_e4m3fn).double() * scales.double().view(1, -1, 1, 1)
+
+
+def pin_fp8_decode_equals_bf16_decode_with_power_of_two_scales():
+    """With power-of-two scales every dequantized value is exactly a bf16, so the FP8
+    decode must equal the bf16 decode of the dequantized cache bit for bit."""
+    w = inputs.make_fp8_decode(3, 8, 2, 300, 32, seed=80, len_range=(0, 300))
+    sl = torch.tensor([0, 1, 300], dtype=torch.int32)
+    ks = torch.tensor([0.125, 4.0], dtype=torch.float32)
+    vs = torch.tensor([2.0, 0.0625], dtype=torch.float32)
+    o, lse = oracle.decode_fp8(w.q, w.kcache, w.vcache, ks, vs, sl, w.scale)
+    kb = _dequant(w.kcache, ks).to(torch.bfloat16)
+    vb = _dequant(w.vcache, vs).to(torch.bfloat16)
+    assert torch.equal(kb.double(), _dequant(w.kcache, ks))
+    ob, lb = oracle.decode(w.q, kb, vb, sl, w.scale)
+    assert torch.equal(o, ob) and torch.equal(lse, lb)
+
+
+def pin_fp8_decode_library_sdpa():
+    """Arbitrary per-head scales: torch fp64 SDPA on the dequantized cache."""
+    w = inputs.make_fp8_decode(2, 8, 4, 200, 64, seed=81, len_range=(1, 200))
+    o, lse = oracle.decode_fp8(w.q, w.kcache, w.vcache, w.k_scale, w.v_scale, w.seqlens, w.scale)
+    assert not torch.equal(w.k_scale, w.v_scale)
+    kd, vd = _dequant(w.kcache, w.k_scale), _dequant(w.vcache, w.v_scale)
+    for b in range(2):
+        L = int(w.seqlens[b])
+        q = w.q[b:b + 1].unsqueeze(2).double()
+        kk = kd[b:b + 1, :, :L].repeat_interleave(2, dim=1)
+        vv = vd[b:b + 1, :, :L].repeat_interleave(2, dim=1)
+        ro = F.scaled_dot_product_attention(q, kk, vv, scale=w.scale)
+        rl = torch.logsumexp(torch.matmul(q, kk.transpose(-1, -2)) * w.scale, dim=-1)
+        assert torch.allclose(o[b], ro[0, :, 0], atol=1e-12, rtol=0)
+        assert torch.allclose(lse[b], rl[0, :, 0], atol=1e-12, rtol=0)
+
+
 PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]
 
 
@@ -390,6 +442,11 @@ MUTANTS = [
     ("paged pool layout", "const long src = ((page * Hkv + g) * page_size + row) * d;",
      "const long src = ((g * num_pages + page) * page_size + row) * d;"),
     ("paged head map", "for (long h = g * R; h < (g + 1) * R; ++h)", "for (long h = g; h < Hq; h += Hkv)"),
+    ("e4m3 bias", "v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("e4m3 subnormal", "v = ldexp((double)m / 8.0, -6);", "v = ldexp((double)m / 8.0, -7);"),
+    ("fp8 scales swapped", "kd[e] = (double)k_scale[g] * oracle_e4m3_to_double(kh[e]);",
+     "kd[e] = (double)v_scale[g] * oracle_e4m3_to_double(kh[e]);"),
+    ("fp8 normaliser dropped", "double w = exp(s[j] - mx) / sum;", "double w = exp(s[j] - mx);"),
 ]
 
 
