@@ -421,8 +421,9 @@ def run_ours(args, rank, world, local):
 
 
 def run_extra(args, dev, peaks):
-    """Per-workload kernel times for the other prefill workloads (not part of the step):
-    the other causal shapes, sliding window (6, 8) and chunked prefill (7, 8)."""
+    """Per-workload kernel times for the other workloads (not part of the step): the other
+    causal shapes, sliding window (6, 8), chunked prefill (7, 8), paged decode (9) and FP8
+    decode (10).  Caches of decode 9 and 10 (over 1 GB) exceed L2; prefill 1 does not."""
     from exact_io_aware_81_b200 import ops
     res = {}
     for kid in (1, 3, 4, 6, 7, 8):
@@ -446,6 +447,39 @@ def run_extra(args, dev, peaks):
         tf = w.flops() / (ms * 1e-3) / 1e12
         res[w.name] = {"ms": ms, "tflops": tf, "frac": tf / peaks.get("bf16_tflops", 1590.0)}
         del q, k, v, o, lse
+        torch.cuda.empty_cache()
+    # decode over a paged cache (9) and over an FP8 cache (10): HBM-bound like decode 5
+    for kid in (9, 10):
+        w = inputs.workload(kid)
+        sl = w.seqlens.to(dev)
+        qd = w.q.to(dev)
+        B, Hq, d = qd.shape
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+        ls = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        if kid == 9:
+            kp, vp, bt = w.kpages.to(dev), w.vpages.to(dev), w.block_table.to(dev)
+            nmax = kp.shape[2] * bt.shape[1]
+            wsp = torch.empty(ops.decode_workspace_size(B, Hq, nmax, d), dtype=torch.uint8, device=dev)
+            run = lambda: ops.decode_paged(qd, kp, vp, bt, sl, scale=w.scale, workspace=wsp, out=out, lse=ls)
+        else:
+            kc, vc = w.kcache.to(dev), w.vcache.to(dev)
+            ks, vs = w.k_scale.to(dev), w.v_scale.to(dev)
+            wsp = torch.empty(ops.decode_workspace_size(B, Hq, kc.shape[2], d), dtype=torch.uint8, device=dev)
+            run = lambda: ops.decode_fp8(qd, kc, vc, ks, vs, sl, scale=w.scale, workspace=wsp, out=out, lse=ls)
+        for _ in range(3):
+            run()
+        n = 20
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record()
+        for _ in range(n):
+            run()
+        e[1].record()
+        torch.cuda.synchronize(dev)
+        ms = e[0].elapsed_time(e[1]) / n
+        gbs = w.io_bytes() / (ms * 1e-3) / 1e9
+        res[w.name] = {"ms": ms, "gbs": gbs, "frac": gbs / peaks.get("hbm_gbs", 6650.0),
+                       "cache_bytes": w.cache_bytes()}
+        del w, run
         torch.cuda.empty_cache()
     assert ops.get_error() == ops.FA_OK
     return res

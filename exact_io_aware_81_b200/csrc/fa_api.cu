@@ -49,7 +49,7 @@ struct DeviceInfo {
     bool sm100 = false;
     int num_sms = 0;
     bool prefill_attr_set[2][2][2][2] = {};
-    bool decode_attr_set[2][4][2] = {};
+    bool decode_attr_set[2][4][2][2] = {};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -102,15 +102,18 @@ EncodeTiledFn get_encode_fn()
 // A (D, rows, planes) bf16 tensor with boxes of `box_rows` rows x 64 columns, 128-byte
 // swizzle.
 int encode_rows_map(CUtensorMap *m, const void *base, int D, long long rows, long long planes,
-                    unsigned box_rows = 128)
+                    unsigned box_rows = 128, bool fp8 = false)
 {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    // one box row is 128 bytes: 64 bf16 or 128 FP8 (byte) elements
+    const cuuint64_t eb = fp8 ? 1 : 2;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
-    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint64_t strides[2] = {(cuuint64_t)D * eb, (cuuint64_t)rows * D * eb};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / eb), box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+    CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void *>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -243,16 +246,16 @@ size_t decode_ws_bytes(int B, int Hq, int Nmax, int d)
 }
 
 // Persistent split kernel: one CTA per SM (at most one per work item).
-template <int D, int RG, bool PAGED>
+template <int D, int RG, bool PAGED, bool FP8>
 int launch_split(fa::DecodeParams p, DeviceInfo *info, cudaStream_t st)
 {
-    using C = fa::decode::SplitCfg<D, RG>;
+    using C = fa::decode::SplitCfg<D, RG, FP8>;
     static_assert(C::kSmemBytes * fa::decode::kCtasPerSm <= 227 * 1024, "decode CTAs per SM do not fit");
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
-        bool &set = info->decode_attr_set[D == 128][RG == 8 ? 3 : RG == 4 ? 2 : RG == 2 ? 1 : 0][PAGED];
+        bool &set = info->decode_attr_set[D == 128][RG == 8 ? 3 : RG == 4 ? 2 : RG == 2 ? 1 : 0][PAGED][FP8];
         if (!set) {
-            cudaError_t e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, RG, PAGED>,
+            cudaError_t e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, RG, PAGED, FP8>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
             if (e != cudaSuccess)
                 return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -263,18 +266,18 @@ int launch_split(fa::DecodeParams p, DeviceInfo *info, cudaStream_t st)
     p.n_items = p.S_max * p.B * p.n_hg;
     const int max_ctas = fa::decode::kCtasPerSm * info->num_sms;
     const int grid = p.n_items < max_ctas ? p.n_items : max_ctas;
-    fa::fa_decode_split_kernel<D, RG, PAGED><<<grid, fa::decode::kThreads, C::kSmemBytes, st>>>(p);
+    fa::fa_decode_split_kernel<D, RG, PAGED, FP8><<<grid, fa::decode::kThreads, C::kSmemBytes, st>>>(p);
     return FA_OK;
 }
 
-template <int D, bool PAGED = false>
+template <int D, bool PAGED = false, bool FP8 = false>
 int launch_split_rg(const fa::DecodeParams &p, int rg, DeviceInfo *info, cudaStream_t st)
 {
     switch (rg) {
-    case 8: return launch_split<D, 8, PAGED>(p, info, st);
-    case 4: return launch_split<D, 4, PAGED>(p, info, st);
-    case 2: return launch_split<D, 2, PAGED>(p, info, st);
-    default: return launch_split<D, 1, PAGED>(p, info, st);
+    case 8: return launch_split<D, 8, PAGED, FP8>(p, info, st);
+    case 4: return launch_split<D, 4, PAGED, FP8>(p, info, st);
+    case 2: return launch_split<D, 2, PAGED, FP8>(p, info, st);
+    default: return launch_split<D, 1, PAGED, FP8>(p, info, st);
     }
 }
 
@@ -385,27 +388,51 @@ int fa_decode(const void *q, const void *kcache, const void *vcache, const int *
     return ok();
 }
 
-int fa_decode_paged(const void *q, const void *kpages, const void *vpages, const int *block_table,
-                    const int *seqlens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
-                    int page_size, int max_pages, int d, float scale, void *workspace,
-                    size_t workspace_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// The caches of a decode call beyond the contiguous bf16 layout of fa_decode.
+struct CacheDesc {
+    const void *k, *v;                // contiguous caches (B, Hkv, Nmax, d) or page pools
+    bool fp8;                         // E4M3 bytes with per-head scales
+    const float *k_scale, *v_scale;   // (Hkv) each, FP8 only
+    bool paged;
+    const int *block_table;           // (B, max_pages), paged only
+    int num_pages, page_size, max_pages;
+};
+
+// Validation and launch shared by the paged and the FP8 entry points.  Nmax is the
+// contiguous cache length (ignored when paged: page_size * max_pages).
+int decode_general(const void *q, const CacheDesc &c, const int *seqlens, void *o, float *lse,
+                   int B, int Hq, int Hkv, int Nmax, int d, float scale, void *workspace,
+                   size_t workspace_bytes, void *stream)
 {
-    if (!q || !kpages || !vpages || !block_table || !seqlens || !o)
-        return fail(FA_ERR_INVALID, "null pointer argument");
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || num_pages <= 0 || page_size <= 0 || max_pages <= 0 || d <= 0)
-        return fail(FA_ERR_INVALID,
-                    "sizes must be positive (B=%d Hq=%d Hkv=%d num_pages=%d page_size=%d max_pages=%d d=%d)",
-                    B, Hq, Hkv, num_pages, page_size, max_pages, d);
+    if (!q || !c.k || !c.v || !seqlens || !o) return fail(FA_ERR_INVALID, "null pointer argument");
+    if (c.fp8 && (!c.k_scale || !c.v_scale)) return fail(FA_ERR_INVALID, "null scale pointer");
+    if (c.paged && !c.block_table) return fail(FA_ERR_INVALID, "null block table");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0)
+        return fail(FA_ERR_INVALID, "sizes must be positive (B=%d Hq=%d Hkv=%d d=%d)", B, Hq, Hkv, d);
+    if (c.paged) {
+        if (c.num_pages <= 0 || c.page_size <= 0 || c.max_pages <= 0)
+            return fail(FA_ERR_INVALID, "page sizes must be positive (num_pages=%d page_size=%d max_pages=%d)",
+                        c.num_pages, c.page_size, c.max_pages);
+    } else if (Nmax <= 0) {
+        return fail(FA_ERR_INVALID, "Nmax must be positive (%d)", Nmax);
+    }
     if (Hq % Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
     if (!(scale > 0.f) || !std::isfinite(scale)) return fail(FA_ERR_INVALID, "scale must be finite and > 0");
     if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
-    if (page_size % 16 != 0) return fail(FA_ERR_UNSUPPORTED, "page_size %d is not a multiple of 16", page_size);
-    if (!aligned16(q) || !aligned16(kpages) || !aligned16(vpages) || !aligned16(o))
-        return fail(FA_ERR_UNSUPPORTED, "q, kpages, vpages and o must be 16-byte aligned");
-    const long long nmax = (long long)page_size * max_pages;
-    if (B > 65535 || nmax > 0x7fffffffLL || (long long)num_pages * Hkv > 0x7fffffffLL)
+    if (c.fp8 && d != 128) return fail(FA_ERR_UNSUPPORTED, "FP8 caches need d = 128 (got %d)", d);
+    if (c.paged && c.page_size % 16 != 0)
+        return fail(FA_ERR_UNSUPPORTED, "page_size %d is not a multiple of 16", c.page_size);
+    if (!aligned16(q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(o))
+        return fail(FA_ERR_UNSUPPORTED, "q, the caches and o must be 16-byte aligned");
+    const long long nmax = c.paged ? (long long)c.page_size * c.max_pages : Nmax;
+    const long long planes = c.paged ? (long long)c.num_pages * Hkv : (long long)B * Hkv;
+    if (B > 65535 || nmax > 0x7fffffffLL || planes > 0x7fffffffLL)
         return fail(FA_ERR_UNSUPPORTED, "problem too large");
-    const int Nmax = (int)nmax;
+    Nmax = (int)nmax;
     const size_t need = decode_ws_bytes(B, Hq, Nmax, d);
     if (!workspace || workspace_bytes < need)
         return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
@@ -420,16 +447,23 @@ int fa_decode_paged(const void *q, const void *kpages, const void *vpages, const
 
     fa::DecodeParams p;
     memset(&p, 0, sizeof p);
-    // rows per copy: the largest power of two that divides page_size, at most 64
-    p.box_rows = page_size & -page_size;
-    if (p.box_rows > fa::decode::kSub) p.box_rows = fa::decode::kSub;
     p.q = static_cast<const __nv_bfloat16 *>(q);
-    if ((rc = encode_rows_map(&p.tm_k, kpages, d, page_size, (long long)num_pages * Hkv, p.box_rows)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_v, vpages, d, page_size, (long long)num_pages * Hkv, p.box_rows)) != FA_OK) return rc;
-    p.block_table = block_table;
-    p.page_size = page_size;
-    p.max_pages = max_pages;
-    p.num_pages = num_pages;
+    if (c.paged) {
+        // rows per copy: the largest power of two that divides page_size, at most 64
+        p.box_rows = c.page_size & -c.page_size;
+        if (p.box_rows > fa::decode::kSub) p.box_rows = fa::decode::kSub;
+        p.block_table = c.block_table;
+        p.page_size = c.page_size;
+        p.max_pages = c.max_pages;
+        p.num_pages = c.num_pages;
+    } else {
+        p.box_rows = fa::decode::kSub;
+    }
+    const long long map_rows = c.paged ? c.page_size : Nmax;
+    if ((rc = encode_rows_map(&p.tm_k, c.k, d, map_rows, planes, p.box_rows, c.fp8)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, c.v, d, map_rows, planes, p.box_rows, c.fp8)) != FA_OK) return rc;
+    p.k_scale = c.k_scale;
+    p.v_scale = c.v_scale;
     p.seqlens = seqlens;
     p.S_max = (int)decode_splits(Nmax);
     p.part_o = static_cast<float *>(workspace);
@@ -446,13 +480,50 @@ int fa_decode_paged(const void *q, const void *kpages, const void *vpages, const
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     p.wait_limit_ns = g_wait_limit_ns;
-    rc = (d == 128) ? launch_split_rg<128, true>(p, rg, info, st) : launch_split_rg<64, true>(p, rg, info, st);
+    if (c.fp8)
+        rc = c.paged ? launch_split_rg<128, true, true>(p, rg, info, st) : launch_split_rg<128, false, true>(p, rg, info, st);
+    else if (c.paged)
+        rc = (d == 128) ? launch_split_rg<128, true>(p, rg, info, st) : launch_split_rg<64, true>(p, rg, info, st);
+    else
+        rc = (d == 128) ? launch_split_rg<128, false>(p, rg, info, st) : launch_split_rg<64, false>(p, rg, info, st);
     if (rc != FA_OK) return rc;
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "paged decode split launch: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
     e = (d == 128) ? launch_merge<128>(p, st) : launch_merge<64>(p, st);
     if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
     return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_decode_paged(const void *q, const void *kpages, const void *vpages, const int *block_table,
+                    const int *seqlens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
+                    int page_size, int max_pages, int d, float scale, void *workspace,
+                    size_t workspace_bytes, void *stream)
+{
+    const CacheDesc c{kpages, vpages, false, nullptr, nullptr, true, block_table, num_pages, page_size, max_pages};
+    return decode_general(q, c, seqlens, o, lse, B, Hq, Hkv, 0, d, scale, workspace, workspace_bytes, stream);
+}
+
+int fa_decode_fp8(const void *q, const void *kcache, const void *vcache, const float *k_scale,
+                  const float *v_scale, const int *seqlens, void *o, float *lse, int B, int Hq,
+                  int Hkv, int Nmax, int d, float scale, void *workspace, size_t workspace_bytes,
+                  void *stream)
+{
+    const CacheDesc c{kcache, vcache, true, k_scale, v_scale, false, nullptr, 0, 0, 0};
+    return decode_general(q, c, seqlens, o, lse, B, Hq, Hkv, Nmax, d, scale, workspace, workspace_bytes, stream);
+}
+
+int fa_decode_paged_fp8(const void *q, const void *kpages, const void *vpages, const float *k_scale,
+                        const float *v_scale, const int *block_table, const int *seqlens, void *o,
+                        float *lse, int B, int Hq, int Hkv, int num_pages, int page_size,
+                        int max_pages, int d, float scale, void *workspace, size_t workspace_bytes,
+                        void *stream)
+{
+    const CacheDesc c{kpages, vpages, true, k_scale, v_scale, true, block_table, num_pages, page_size, max_pages};
+    return decode_general(q, c, seqlens, o, lse, B, Hq, Hkv, 0, d, scale, workspace, workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------ allocation-free decode

@@ -25,10 +25,26 @@
 // physical pages of an item's keys in the block table (one entry per lane) and copies
 // boxes of box_rows rows, a power of two that divides page_size, so no box straddles two
 // pages; the consumers and the merge are unchanged.
+//
+// FP8 caches (E4M3 bytes with one dequantization scale per K/V head for K and one for V;
+// youngju.dev sections 5 and 7 name FP8 KV caches) halve the bytes read.  Each E4M3 pair
+// is converted exactly to fp16 in registers and the same mma.sync tiles run on fp16
+// operands:
+//   K pass: ldmatrix (not transposed) hands a lane 4 consecutive dims of one key; the
+//     MMA's contraction index is permuted so that those 4 dims are the lane's two B
+//     registers, and q is loaded in the same permuted order (so no transpose is needed).
+//     q is scaled per row by an exact power of two 2^e so that its largest element lies
+//     in [2^14, 2^15) before the fp16 conversion (every bf16 value in that range is an
+//     fp16 value); the factor k_scale * 2^-e is applied to the fp32 scores.
+//   V pass: a transposing 16-bit ldmatrix hands a lane 2 dims x 2 keys; one byte permute
+//     splits them into the key pairs of an even and an odd dim, which are the B
+//     registers of two MMAs whose output columns are the even and the odd dims.  P is
+//     converted to fp16 and v_scale is applied with the final 1 / l.
 #pragma once
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "fa_common.cuh"
 #include "ptx_sm100.cuh"
@@ -50,6 +66,8 @@ struct DecodeParams {
     int n_items;   // S_max * B * n_hg candidate work items (chunk-major order)
     float scale_log2;
     unsigned long long wait_limit_ns;
+    // FP8 cache only: per K/V head dequantization scales (Hkv each)
+    const float *k_scale, *v_scale;
     // paged cache only (Nmax = page_size * max_pages)
     const int *block_table;   // (B, max_pages) physical page of each logical page
     int page_size, max_pages, num_pages;
@@ -66,10 +84,13 @@ constexpr int kCtasPerSm = 3;
 constexpr int kBoxBytes = kSub * 128;  // 64 rows x 64 bf16 columns
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int D, int RG>
+template <int D, int RG, bool FP8>
 struct SplitCfg {
-    static constexpr int kStageBytes = (D / 64) * kBoxBytes;
-    static constexpr int kStages = (D == 128) ? 4 : 8;                 // 64 KB ring
+    static constexpr int kEB = FP8 ? 1 : 2;                            // bytes per cache element
+    static constexpr int kColBoxes = D * kEB / 128;                    // 128-byte column boxes per row
+    static constexpr int kRowChunks = D * kEB / 16;                    // 16-byte chunks per row
+    static constexpr int kStageBytes = kColBoxes * kBoxBytes;
+    static constexpr int kStages = (kStageBytes == 2 * kBoxBytes) ? 4 : 8;  // 64 KB ring
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kScoreOff = kRingBytes;                       // float [RG][kChunk]
     static constexpr int kMOff = kScoreOff + RG * kChunk * 4;          // float m[RG], l[RG]
@@ -92,6 +113,13 @@ __device__ __forceinline__ uint32_t stage_offset(int r, int c)
 }
 
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) { return ptx::pack_bf16x2(lo, hi); }
+
+// Two E4M3 bytes (low byte -> low half) to packed fp16; exact for every finite E4M3 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes)
+{
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_bytes & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
 
 }  // namespace decode
 
@@ -117,13 +145,14 @@ __device__ __forceinline__ bool decode_item(const DecodeParams &p, int it, int &
 // (rows RG .. 15 are zero): S = Q K^T per 8-key column tile, O += P V per 8-column tile,
 // both with fp32 accumulation; K and V fragments come from the swizzled stages through
 // ldmatrix (transposed for V).
-template <int D, int RG, bool PAGED>
+template <int D, int RG, bool PAGED, bool FP8>
 __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
     fa_decode_split_kernel(const __grid_constant__ DecodeParams p)
 {
     using namespace decode;
-    using C = SplitCfg<D, RG>;
+    using C = SplitCfg<D, RG, FP8>;
     static_assert(RG <= 8, "at most 8 query heads per item");
+    static_assert(!FP8 || D == 128, "FP8 caches: d = 128 (one 128-byte row per key)");
     constexpr int KSTEPS = D / 16;          // k-steps of S = Q K^T
     constexpr int NT = D / 8 / kWarps;      // 8-column tiles of O per consumer warp
 
@@ -199,25 +228,25 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                         // only the boxes that hold keys of the sequence are copied (rows past
                         // it are masked or cleared by the consumers)
                         const int nbox = (min(kSub, n - t * kSub) + p.box_rows - 1) / p.box_rows;
-                        if (leader) ptx::mbar_arrive_expect_tx(&full[st], nbox * p.box_rows * 128 * (D / 64));
+                        if (leader) ptx::mbar_arrive_expect_tx(&full[st], nbox * p.box_rows * 128 * C::kColBoxes);
                         for (int i = 0; i < nbox; ++i) {
                             const int key = start + t * kSub + i * p.box_rows;
                             const int lp = key / p.page_size;
                             const int page = __shfl_sync(0xffffffffu, my_page, lp - first_lp);
                             if (leader) {
 #pragma unroll
-                                for (int c = 0; c < D / 64; ++c)
+                                for (int c = 0; c < C::kColBoxes; ++c)
                                     ptx::tma_load_3d(smem + st * C::kStageBytes + c * kBoxBytes + i * p.box_rows * 128,
-                                                     map, &full[st], 64 * c, key - lp * p.page_size,
+                                                     map, &full[st], c * (128 / C::kEB), key - lp * p.page_size,
                                                      page * p.Hkv + g);
                             }
                         }
                     } else if (leader) {
                         ptx::mbar_arrive_expect_tx(&full[st], C::kStageBytes);
 #pragma unroll
-                        for (int c = 0; c < D / 64; ++c)
+                        for (int c = 0; c < C::kColBoxes; ++c)
                             ptx::tma_load_3d(smem + st * C::kStageBytes + c * kBoxBytes, map, &full[st],
-                                             64 * c, start + t * kSub, plane);
+                                             c * (128 / C::kEB), start + t * kSub, plane);
                     }
                     __syncwarp();
                     ++ring;
@@ -249,14 +278,50 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             int b, hg, start, n;
             if (!decode_item(p, it, b, hg, start, n)) continue;
             const int h0 = hg * RG;
-            // A operand of S = Q K^T: row gid = query head h0 + gid (zero beyond RG)
+            const int g = h0 / p.R;
+            // A operand of S = Q K^T: row gid = query head h0 + gid (zero beyond RG).
+            // bf16: K step ks holds dims 16ks + 2tig + {0,1} and 16ks + 8 + 2tig + {0,1}.
+            // FP8:  K step ks holds dims 16ks + 4tig + {0,1} and 16ks + 4tig + {2,3} (the
+            //       permuted contraction order of the K pass), as fp16 scaled by 2^e.
             uint32_t qa[KSTEPS][2];
+            float sl_row = p.scale_log2;  // factor from the MMA result to log2-domain scores
             {
-                const uint32_t *qrow = reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + h0 + (row_real ? gid : 0)) * D);
+                const __nv_bfloat16 *qrow = p.q + ((size_t)b * p.Hq + h0 + (row_real ? gid : 0)) * D;
+                if constexpr (FP8) {
+                    float qv[KSTEPS][4];
+                    float amax = 0.f;
 #pragma unroll
-                for (int ks = 0; ks < KSTEPS; ++ks) {
-                    qa[ks][0] = row_real ? qrow[8 * ks + tig] : 0u;
-                    qa[ks][1] = row_real ? qrow[8 * ks + 4 + tig] : 0u;
+                    for (int ks = 0; ks < KSTEPS; ++ks) {
+                        const uint2 raw = row_real ? *reinterpret_cast<const uint2 *>(qrow + 16 * ks + 4 * tig)
+                                                   : make_uint2(0u, 0u);
+                        qv[ks][0] = __uint_as_float(raw.x << 16);
+                        qv[ks][1] = __uint_as_float(raw.x & 0xffff0000u);
+                        qv[ks][2] = __uint_as_float(raw.y << 16);
+                        qv[ks][3] = __uint_as_float(raw.y & 0xffff0000u);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qv[ks][e]));
+                    }
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                    // 2^e with amax * 2^e in [2^14, 2^15); e kept within the normal range
+                    int e = 0;
+                    if (amax > 0.f) e = 14 - (((int)(__float_as_uint(amax) >> 23) & 0xff) - 127);
+                    e = max(-120, min(120, e));
+                    const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+                    const float down = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+                    for (int ks = 0; ks < KSTEPS; ++ks) {
+                        qa[ks][0] = ptx::pack_f16x2(qv[ks][0] * up, qv[ks][1] * up);
+                        qa[ks][1] = ptx::pack_f16x2(qv[ks][2] * up, qv[ks][3] * up);
+                    }
+                    sl_row = p.scale_log2 * p.k_scale[g] * down;
+                } else {
+                    const uint32_t *qw = reinterpret_cast<const uint32_t *>(qrow);
+#pragma unroll
+                    for (int ks = 0; ks < KSTEPS; ++ks) {
+                        qa[ks][0] = row_real ? qw[8 * ks + tig] : 0u;
+                        qa[ks][1] = row_real ? qw[8 * ks + 4 + tig] : 0u;
+                    }
                 }
             }
             bool ok = true;
@@ -269,19 +334,35 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                 for (int nt = 0; nt < 2; ++nt) {
                     const int key0 = warp * 16 + nt * 8;  // 8 keys of this column tile
                     float c[4] = {0.f, 0.f, 0.f, 0.f};
+                    if constexpr (FP8) {
+                        // matrix m of a load: 16-byte chunk 4 * half + m of the 8 keys' rows;
+                        // the lane's register = dims 4tig .. 4tig+3 of key gid in that chunk
 #pragma unroll
-                    for (int ks = 0; ks < KSTEPS; ks += 2) {
-                        uint32_t b0, b1, b2, b3;
-                        ptx::ldsm_x4(sbase + stage_offset(key0 + lm_row, 2 * ks + lm_mat), b0, b1, b2, b3);
-                        const uint32_t a0[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
-                        const uint32_t a1[4] = {qa[ks + 1][0], 0u, qa[ks + 1][1], 0u};
-                        ptx::mma_16816_bf16(c, a0, b0, b1);
-                        ptx::mma_16816_bf16(c, a1, b2, b3);
+                        for (int half = 0; half < 2; ++half) {
+                            uint32_t r[4];
+                            ptx::ldsm_x4(sbase + stage_offset(key0 + lm_row, 4 * half + lm_mat), r[0], r[1], r[2], r[3]);
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {
+                                const int ks = 4 * half + m;
+                                const uint32_t a[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
+                                ptx::mma_16816_f16(c, a, e4m3x2_to_f16x2(r[m]), e4m3x2_to_f16x2(r[m] >> 16));
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ks += 2) {
+                            uint32_t b0, b1, b2, b3;
+                            ptx::ldsm_x4(sbase + stage_offset(key0 + lm_row, 2 * ks + lm_mat), b0, b1, b2, b3);
+                            const uint32_t a0[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
+                            const uint32_t a1[4] = {qa[ks + 1][0], 0u, qa[ks + 1][1], 0u};
+                            ptx::mma_16816_bf16(c, a0, b0, b1);
+                            ptx::mma_16816_bf16(c, a1, b2, b3);
+                        }
                     }
                     if (row_real) {
                         const int key = t * kSub + key0 + 2 * tig;
-                        s_sm[gid][key] = key < n ? c[0] * p.scale_log2 : -INFINITY;
-                        s_sm[gid][key + 1] = key + 1 < n ? c[1] * p.scale_log2 : -INFINITY;
+                        s_sm[gid][key] = key < n ? c[0] * sl_row : -INFINITY;
+                        s_sm[gid][key + 1] = key + 1 < n ? c[1] * sl_row : -INFINITY;
                     }
                 }
                 __syncwarp();
@@ -310,6 +391,8 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             }
             if (!gb.sync(sf)) break;
             // ------------------------------------------------------------ V pass
+            // bf16: acc[j] = column tile warp * NT + j (8 dims).  FP8: acc[2 * blk + par]
+            // holds the even (par 0) / odd (par 1) dims of 16-dim block 2 * warp + blk.
             float acc[NT][4];
 #pragma unroll
             for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
@@ -319,12 +402,13 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                 uint8_t *stage = smem + st * C::kStageBytes;
                 const int rows = min(kSub, n - t * kSub);
                 if (rows < kSub) {
-                    // rows past the sequence hold whatever the cache holds there: clear them
-                    // so that their zero weights cannot meet a non-finite value (and order
-                    // these writes before the copy engine refills the stage)
-                    for (int idx = threadIdx.x; idx < (kSub - rows) * (D / 8); idx += 32 * kWarps) {
-                        const int r = rows + idx / (D / 8);
-                        *reinterpret_cast<uint4 *>(stage + stage_offset(r, idx % (D / 8))) = make_uint4(0, 0, 0, 0);
+                    // rows past the sequence hold whatever the cache holds there (or, paged,
+                    // an earlier stage's data): clear them so that their zero weights cannot
+                    // meet a non-finite value (and order these writes before the copy engine
+                    // refills the stage)
+                    for (int idx = threadIdx.x; idx < (kSub - rows) * C::kRowChunks; idx += 32 * kWarps) {
+                        const int r = rows + idx / C::kRowChunks;
+                        *reinterpret_cast<uint4 *>(stage + stage_offset(r, idx % C::kRowChunks)) = make_uint4(0, 0, 0, 0);
                     }
                     ptx::fence_proxy_async_smem();
                     if (!gb.sync(sf)) { ok = false; break; }
@@ -332,23 +416,44 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                 const uint32_t sbase = ptx::smem_addr(stage);
 #pragma unroll
                 for (int kb = 0; kb < kSub; kb += 16) {
-                    // A operand: P of row gid for keys kb .. kb+15 (bf16), zero beyond RG
+                    // A operand: P of row gid for keys kb .. kb+15, zero beyond RG
                     uint32_t pa[4] = {0u, 0u, 0u, 0u};
                     if (row_real) {
                         const float2 p0 = *reinterpret_cast<const float2 *>(&s_sm[gid][t * kSub + kb + 2 * tig]);
                         const float2 p1 = *reinterpret_cast<const float2 *>(&s_sm[gid][t * kSub + kb + 8 + 2 * tig]);
-                        pa[0] = pack2_bf16(p0.x, p0.y);
-                        pa[2] = pack2_bf16(p1.x, p1.y);
+                        if constexpr (FP8) {
+                            pa[0] = ptx::pack_f16x2(p0.x, p0.y);
+                            pa[2] = ptx::pack_f16x2(p1.x, p1.y);
+                        } else {
+                            pa[0] = pack2_bf16(p0.x, p0.y);
+                            pa[2] = pack2_bf16(p1.x, p1.y);
+                        }
                     }
+                    if constexpr (FP8) {
+                        // matrices: (keys kb..+7 | kb+8..+15) x (16-dim block 2 * warp | + 1);
+                        // a lane gets bytes {V[2tig][2gid], V[2tig][2gid+1], V[2tig+1][2gid],
+                        // V[2tig+1][2gid+1]} of its matrix
+                        uint32_t r[4];
+                        ptx::ldsm_x4_trans(sbase + stage_offset(kb + (lm_mat & 1) * 8 + lm_row, 2 * warp + (lm_mat >> 1)),
+                                           r[0], r[1], r[2], r[3]);
 #pragma unroll
-                    for (int j = 0; j < NT; j += 2) {
-                        // matrices: (keys kb..+7 | kb+8..+15) x (column tile j | j+1)
-                        const int chunk = (warp * NT + j) + (lm_mat >> 1);
-                        const int row = kb + (lm_mat & 1) * 8 + lm_row;
-                        uint32_t b0, b1, b2, b3;
-                        ptx::ldsm_x4_trans(sbase + stage_offset(row, chunk), b0, b1, b2, b3);
-                        ptx::mma_16816_bf16(acc[j], pa, b0, b1);
-                        ptx::mma_16816_bf16(acc[j + 1], pa, b2, b3);
+                        for (int blk = 0; blk < 2; ++blk) {
+                            const uint32_t lo = __byte_perm(r[2 * blk], 0u, 0x3120);      // keys kb + 2tig, +1
+                            const uint32_t hi = __byte_perm(r[2 * blk + 1], 0u, 0x3120);  // keys kb + 8 + 2tig, +1
+                            ptx::mma_16816_f16(acc[2 * blk], pa, e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi));
+                            ptx::mma_16816_f16(acc[2 * blk + 1], pa, e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi >> 16));
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < NT; j += 2) {
+                            // matrices: (keys kb..+7 | kb+8..+15) x (column tile j | j+1)
+                            const int chunk = (warp * NT + j) + (lm_mat >> 1);
+                            const int row = kb + (lm_mat & 1) * 8 + lm_row;
+                            uint32_t b0, b1, b2, b3;
+                            ptx::ldsm_x4_trans(sbase + stage_offset(row, chunk), b0, b1, b2, b3);
+                            ptx::mma_16816_bf16(acc[j], pa, b0, b1);
+                            ptx::mma_16816_bf16(acc[j + 1], pa, b2, b3);
+                        }
                     }
                 }
                 __syncwarp();
@@ -358,12 +463,25 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             if (!ok) break;
             const int chunk = start / kChunk;
             if (row_real) {
-                const float inv_l = 1.f / l_sm[gid];
                 float *dst = p.part_o + (((size_t)b * p.Hq + h0 + gid) * p.S_max + chunk) * D;
+                if constexpr (FP8) {
+                    const float f = p.v_scale[g] / l_sm[gid];
 #pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    const int col = (warp * NT + j) * 8 + 2 * tig;
-                    *reinterpret_cast<float2 *>(dst + col) = make_float2(acc[j][0] * inv_l, acc[j][1] * inv_l);
+                    for (int blk = 0; blk < 2; ++blk) {
+                        // acc[2blk] columns 2tig, 2tig+1 = dims 4tig, 4tig+2 of the block;
+                        // acc[2blk+1] the odd dims 4tig+1, 4tig+3
+                        const int col = (2 * warp + blk) * 16 + 4 * tig;
+                        *reinterpret_cast<float4 *>(dst + col) =
+                            make_float4(acc[2 * blk][0] * f, acc[2 * blk + 1][0] * f,
+                                        acc[2 * blk][1] * f, acc[2 * blk + 1][1] * f);
+                    }
+                } else {
+                    const float inv_l = 1.f / l_sm[gid];
+#pragma unroll
+                    for (int j = 0; j < NT; ++j) {
+                        const int col = (warp * NT + j) * 8 + 2 * tig;
+                        *reinterpret_cast<float2 *>(dst + col) = make_float2(acc[j][0] * inv_l, acc[j][1] * inv_l);
+                    }
                 }
             }
             if (threadIdx.x < RG)

@@ -38,6 +38,9 @@ SIGNATURES = {
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "fa_decode_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "fa_decode_paged_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
+                                 _P, _Z, _P]),
     "fa_get_error": (_I, [_P]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "fa_fwd_selftest_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
@@ -244,6 +247,92 @@ def decode_paged(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor,
                                 num_pages, page_size, max_pages, d, float(scale),
                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                 _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def _decode_outputs(q, out, lse, want_lse):
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    else:
+        _require(out, "out", torch.bfloat16, 3)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _require(lse, "lse", torch.float32, 2)
+    return out, lse
+
+
+def _workspace(workspace, need, device):
+    if workspace is None:
+        return torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace
+
+
+def decode_fp8(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, k_scale: torch.Tensor,
+               v_scale: torch.Tensor, seqlens: torch.Tensor, scale: Optional[float] = None,
+               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+               lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
+    """Decode over an FP8 E4M3 cache (fa_decode_fp8): kcache/vcache uint8 (B,Hkv,Nmax,d)
+    holding E4M3 bytes; k_scale/v_scale float32 (Hkv,) per-head dequantization scales."""
+    _require(q, "q", torch.bfloat16, 3)
+    _require(kcache, "kcache", torch.uint8, 4)
+    _require(vcache, "vcache", torch.uint8, 4)
+    _require(k_scale, "k_scale", torch.float32, 1)
+    _require(v_scale, "v_scale", torch.float32, 1)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, d = q.shape
+    Bk, Hkv, Nmax, dk = kcache.shape
+    if ((Bk, dk) != (B, d) or tuple(vcache.shape) != tuple(kcache.shape) or seqlens.shape[0] != B
+            or k_scale.shape[0] != Hkv or v_scale.shape[0] != Hkv):
+        raise ValueError("shape mismatch between q, the caches, the scales and seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    workspace = _workspace(workspace, decode_workspace_size(B, Hq, Nmax, d), q.device)
+    out, lse = _decode_outputs(q, out, lse, want_lse)
+    rc = load().fa_decode_fp8(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), k_scale.data_ptr(),
+                              v_scale.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
+                              lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nmax, d,
+                              float(scale), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def decode_paged_fp8(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor,
+                     k_scale: torch.Tensor, v_scale: torch.Tensor, block_table: torch.Tensor,
+                     seqlens: torch.Tensor, scale: Optional[float] = None,
+                     workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
+    """FP8 decode over a paged cache (fa_decode_paged_fp8): pools uint8
+    (num_pages,Hkv,page_size,d) of E4M3 bytes, per-head scales, block table as decode_paged."""
+    _require(q, "q", torch.bfloat16, 3)
+    _require(kpages, "kpages", torch.uint8, 4)
+    _require(vpages, "vpages", torch.uint8, 4)
+    _require(k_scale, "k_scale", torch.float32, 1)
+    _require(v_scale, "v_scale", torch.float32, 1)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, d = q.shape
+    num_pages, Hkv, page_size, dk = kpages.shape
+    max_pages = block_table.shape[1]
+    if (dk != d or tuple(vpages.shape) != tuple(kpages.shape) or seqlens.shape[0] != B
+            or block_table.shape[0] != B or k_scale.shape[0] != Hkv or v_scale.shape[0] != Hkv):
+        raise ValueError("shape mismatch between q, the pools, the scales, block_table and seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    workspace = _workspace(workspace, decode_workspace_size(B, Hq, page_size * max_pages, d), q.device)
+    out, lse = _decode_outputs(q, out, lse, want_lse)
+    rc = load().fa_decode_paged_fp8(q.data_ptr(), kpages.data_ptr(), vpages.data_ptr(),
+                                    k_scale.data_ptr(), v_scale.data_ptr(), block_table.data_ptr(),
+                                    seqlens.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr() if lse is not None else None, B, Hq, Hkv,
+                                    num_pages, page_size, max_pages, d, float(scale),
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    _stream_handle(stream))
     _check(rc)
     return out, lse
 

@@ -140,6 +140,38 @@ FA_API int fa_decode_paged(const void *q, const void *kpages, const void *vpages
                     void *stream);
 
 /*
+ * Decode step over an FP8 KV cache (youngju.dev "attention variants", sections 5 and 7:
+ * storing the cache in FP8 halves its bytes, and decode is bound by reading them).  The
+ * pages fix no scale convention; this library's is one dequantization scale per K/V head
+ * for K and one for V:
+ *   kcache, vcache  (B, Hkv, Nmax, d) bytes, each an OCP FP8 E4M3 ("e4m3fn") value;
+ *   k_scale, v_scale float32[Hkv] in device memory: key j of head g is
+ *                   k_scale[g] * e4m3(kcache[b, g, j, :]), likewise V with v_scale
+ *                   (a single per-tensor scale is the case of equal entries).
+ * q (bf16), o (bf16), lse, seqlens, workspace (fa_decode_workspace_size(B, Hq, Nmax, d)),
+ * scale and stream are those of fa_decode, and so is the result on the dequantized cache.
+ * Supported: d = 128 (FA_ERR_UNSUPPORTED otherwise).  Inside, every E4M3 value is
+ * converted exactly to fp16 and multiplied with fp16 operands (fp32 accumulation); q
+ * enters as fp16 after an exact power-of-two scaling of each row, and the softmax
+ * weights P as fp16.
+ */
+FA_API int fa_decode_fp8(const void *q, const void *kcache, const void *vcache,
+                  const float *k_scale, const float *v_scale, const int *seqlens, void *o,
+                  float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The FP8 decode over a paged cache: kpages/vpages (num_pages, Hkv, page_size, d) E4M3
+ * bytes with the page layout and block table of fa_decode_paged, and the per-head scales
+ * of fa_decode_fp8.  Workspace: fa_decode_workspace_size(B, Hq, page_size * max_pages, d).
+ */
+FA_API int fa_decode_paged_fp8(const void *q, const void *kpages, const void *vpages,
+                        const float *k_scale, const float *v_scale, const int *block_table,
+                        const int *seqlens, void *o, float *lse, int B, int Hq, int Hkv,
+                        int num_pages, int page_size, int max_pages, int d, float scale,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Decode step that allocates nothing and takes no workspace (no counterpart on the
  * pages: an addition of this library for callers that cannot hand it device scratch).
  * Some callers have no way to allocate device memory at the point of the call: plugins

@@ -175,3 +175,37 @@ def _paged(lib, **kw):
 ])
 def test_decode_paged_rejects(lib, kw, status):
     assert _paged(lib, **kw) == status
+
+
+def _fp8(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, ks=FAKE, vs=FAKE, sl=FAKE, o=FAKE, lse=None, B=2, Hq=8, Hkv=2,
+             Nmax=300, d=128, scale=0.1, ws=FAKE, wsb=None)
+    a.update(kw)
+    if a["wsb"] is None:
+        a["wsb"] = lib.fa_decode_workspace_size(a["B"], a["Hq"], a["Nmax"], a["d"])
+    return lib.fa_decode_fp8(a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["sl"], a["o"], a["lse"],
+                             a["B"], a["Hq"], a["Hkv"], a["Nmax"], a["d"], a["scale"], a["ws"],
+                             a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ks=None), ops.FA_ERR_INVALID),
+    (dict(vs=None), ops.FA_ERR_INVALID),
+    (dict(kc=None), ops.FA_ERR_INVALID),
+    (dict(Nmax=0), ops.FA_ERR_INVALID),
+    (dict(Hq=8, Hkv=3), ops.FA_ERR_INVALID),
+    (dict(d=64), ops.FA_ERR_UNSUPPORTED),            # FP8 rows are one 128-byte box
+    (dict(kc=FAKE + 4), ops.FA_ERR_UNSUPPORTED),
+    (dict(wsb=16), ops.FA_ERR_WORKSPACE),
+])
+def test_decode_fp8_rejects(lib, kw, status):
+    assert _fp8(lib, **kw) == status
+
+
+def test_decode_paged_fp8_rejects(lib):
+    rc = lib.fa_decode_paged_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, 2, 8, 2, 10,
+                                 64, 5, 128, 0.1, FAKE, 1 << 20, None)
+    assert rc == ops.FA_ERR_INVALID                  # no block table
+    rc = lib.fa_decode_paged_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 10,
+                                 40, 5, 128, 0.1, FAKE, 1 << 20, None)
+    assert rc == ops.FA_ERR_UNSUPPORTED              # page size not a multiple of 16
