@@ -63,7 +63,7 @@ struct DecodeParams {
     float *lse;               // (B, Hq) natural log, may be null
     int B, Hq, Hkv, Nmax, R, S_max;
     int n_hg;      // head groups: Hq / RG
-    int n_items;   // S_max * B * n_hg candidate work items (chunk-major order)
+    int n_items;   // S_max * B * n_hg: an upper bound on the work items (sizes the grid)
     float scale_log2;
     unsigned long long wait_limit_ns;
     // FP8 cache only: per K/V head dequantization scales (Hkv each)
@@ -123,21 +123,68 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes)
 
 }  // namespace decode
 
-// Work item `it` (chunk-major: the early chunks, valid for every sequence, come first, so
-// a round-robin over the persistent CTAs gives each a similar mix): returns false if the
-// chunk starts past the sequence's length.
-__device__ __forceinline__ bool decode_item(const DecodeParams &p, int it, int &b, int &hg, int &start, int &n)
+// Work items.  Only the valid items are enumerated -- (sequence b, chunk c < ceil(L_b /
+// kChunk), head group hg), sequence-major with the head group fastest -- and item v goes to
+// CTA v mod gridDim.x, so every CTA gets the same number of items to within one whatever
+// the lengths.  The item -> (b, chunk) map needs the prefix sums of the chunk counts; each
+// warp that walks the items keeps a cursor on the sequence of its current item and moves it
+// forward 32 sequences per step (a warp scan of their chunk counts).  Every call below is
+// made by all 32 lanes of a warp with warp-uniform arguments.
+__device__ __forceinline__ int seq_chunks(const DecodeParams &p, int b)
 {
-    const int bh = p.B * p.n_hg;
-    const int chunk = it / bh;
-    const int rest = it - chunk * bh;
-    b = rest / p.n_hg;
-    hg = rest - b * p.n_hg;
+    return (decode::clamp_len(p.seqlens[b], p.Nmax) + decode::kChunk - 1) / decode::kChunk;
+}
+
+// Number of valid items of the launch.
+__device__ __forceinline__ int count_items(const DecodeParams &p)
+{
+    const int lane = threadIdx.x & 31;
+    int s = 0;
+    for (int b = lane; b < p.B; b += 32) s += seq_chunks(p, b);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    return s * p.n_hg;
+}
+
+struct ItemCursor {
+    int b = -1;    // sequence of the last item found
+    int base = 0;  // chunks of the sequences before b
+    int s_b = 0;   // chunks of sequence b
+};
+
+// Item v (< count_items) -> sequence b, head group hg, first key and key count.
+__device__ __forceinline__ void decode_item(const DecodeParams &p, ItemCursor &c, int v, int &b, int &hg,
+                                            int &start, int &n)
+{
+    const int lane = threadIdx.x & 31;
+    const int u = v / p.n_hg;  // index of (b, chunk) in sequence-major order
+    hg = v - u * p.n_hg;
+    if (u >= c.base + c.s_b) {
+        int base = c.base + c.s_b, bb = c.b + 1;
+        while (bb < p.B) {
+            const int sb = (bb + lane < p.B) ? seq_chunks(p, bb + lane) : 0;
+            int incl = sb;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += t;
+            }
+            const unsigned hit = __ballot_sync(0xffffffffu, base + incl > u);
+            if (hit) {
+                const int l = __ffs(hit) - 1;
+                c.b = bb + l;
+                c.s_b = __shfl_sync(0xffffffffu, sb, l);
+                c.base = base + __shfl_sync(0xffffffffu, incl, l) - c.s_b;
+                break;
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
+            bb += 32;
+        }
+    }
+    b = c.b;
     const int L = decode::clamp_len(p.seqlens[b], p.Nmax);
-    start = chunk * decode::kChunk;
-    if (start >= L) return false;
+    start = (u - c.base) * decode::kChunk;
     n = min(decode::kChunk, L - start);
-    return true;
 }
 
 // Split kernel.  D: head dim (64 or 128).  RG: query heads per work item (<= 8, all of one
@@ -154,7 +201,8 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
     static_assert(RG <= 8, "at most 8 query heads per item");
     static_assert(!FP8 || D == 128, "FP8 caches: d = 128 (one 128-byte row per key)");
     constexpr int KSTEPS = D / 16;          // k-steps of S = Q K^T
-    constexpr int NT = D / 8 / kWarps;      // 8-column tiles of O per consumer warp
+    constexpr int VT = D / 16 / kWarps;     // 16-dim tiles of O^T per consumer warp
+    static_assert(VT >= 1 && (!FP8 || VT == 2), "head dims per consumer warp");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -197,9 +245,11 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
         }
         uint32_t ring = 0;
         bool ok = true;
-        for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+        const int n_items = count_items(p);
+        ItemCursor cur;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
             int b, hg, start, n;
-            if (!decode_item(p, it, b, hg, start, n)) continue;
+            decode_item(p, cur, it, b, hg, start, n);
             const int g = hg * RG / p.R;
             const int plane = b * p.Hkv + g;
             // paged: lane i holds the physical page of the item's i-th logical page (an
@@ -274,17 +324,22 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
         // ldmatrix addressing: lane supplies row (lane & 7) of matrix (lane >> 3)
         const int lm_row = lane & 7;
         const int lm_mat = lane >> 3;
-        for (int it = blockIdx.x; it < p.n_items; it += gridDim.x) {
+        const int n_items = count_items(p);
+        ItemCursor cur;
+        for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
             int b, hg, start, n;
-            if (!decode_item(p, it, b, hg, start, n)) continue;
+            decode_item(p, cur, it, b, hg, start, n);
             const int h0 = hg * RG;
             const int g = h0 / p.R;
-            // A operand of S = Q K^T: row gid = query head h0 + gid (zero beyond RG).
+            // The MMAs put the query heads in the N = 8 dimension (RG <= 8) and keys (K pass)
+            // or head dims (V pass) in M = 16, so no MMA row is padding.
+            // B operand of S^T = K Q^T: column gid = query head h0 + gid (zero beyond RG).
             // bf16: K step ks holds dims 16ks + 2tig + {0,1} and 16ks + 8 + 2tig + {0,1}.
             // FP8:  K step ks holds dims 16ks + 4tig + {0,1} and 16ks + 4tig + {2,3} (the
             //       permuted contraction order of the K pass), as fp16 scaled by 2^e.
-            uint32_t qa[KSTEPS][2];
-            float sl_row = p.scale_log2;  // factor from the MMA result to log2-domain scores
+            uint32_t qb[KSTEPS][2];
+            // factors from the MMA result to log2-domain scores of heads 2tig and 2tig+1
+            float sl0 = p.scale_log2, sl1 = p.scale_log2;
             {
                 const __nv_bfloat16 *qrow = p.q + ((size_t)b * p.Hq + h0 + (row_real ? gid : 0)) * D;
                 if constexpr (FP8) {
@@ -311,59 +366,67 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                     const float down = __uint_as_float((uint32_t)(127 - e) << 23);
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks) {
-                        qa[ks][0] = ptx::pack_f16x2(qv[ks][0] * up, qv[ks][1] * up);
-                        qa[ks][1] = ptx::pack_f16x2(qv[ks][2] * up, qv[ks][3] * up);
+                        qb[ks][0] = ptx::pack_f16x2(qv[ks][0] * up, qv[ks][1] * up);
+                        qb[ks][1] = ptx::pack_f16x2(qv[ks][2] * up, qv[ks][3] * up);
                     }
-                    sl_row = p.scale_log2 * p.k_scale[g] * down;
+                    const float sl_own = p.scale_log2 * p.k_scale[g] * down;  // head gid
+                    sl0 = __shfl_sync(0xffffffffu, sl_own, 8 * tig);          // head 2tig
+                    sl1 = __shfl_sync(0xffffffffu, sl_own, 8 * tig + 4);      // head 2tig+1
                 } else {
                     const uint32_t *qw = reinterpret_cast<const uint32_t *>(qrow);
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks) {
-                        qa[ks][0] = row_real ? qw[8 * ks + tig] : 0u;
-                        qa[ks][1] = row_real ? qw[8 * ks + 4 + tig] : 0u;
+                        qb[ks][0] = row_real ? qw[8 * ks + tig] : 0u;
+                        qb[ks][1] = row_real ? qw[8 * ks + 4 + tig] : 0u;
                     }
                 }
             }
+            const int hc0 = 2 * tig, hc1 = 2 * tig + 1;  // the heads of this lane's C columns
             bool ok = true;
             // ------------------------------------------------------------ K pass
+            // warp w: S^T for keys 16w .. 16w+15 of each stage (A = 16 key rows of K)
             for (int t = 0; t * kSub < n; ++t) {
                 const uint32_t st = ring % C::kStages;
                 if (!wait_warp(&full[st], (ring / C::kStages) & 1u, sf)) { ok = false; break; }
                 const uint32_t sbase = ptx::smem_addr(smem + st * C::kStageBytes);
+                const int key0 = warp * 16;
+                // two accumulators (even and odd K steps) halve the dependent MMA chain
+                float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                if constexpr (FP8) {
+                    // matrices: (keys 0-7 | 8-15) x (16-byte chunk 2j | 2j+1); a lane's register
+                    // = dims 4tig .. 4tig+3 of key gid (or gid + 8) of that chunk
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const int key0 = warp * 16 + nt * 8;  // 8 keys of this column tile
-                    float c[4] = {0.f, 0.f, 0.f, 0.f};
-                    if constexpr (FP8) {
-                        // matrix m of a load: 16-byte chunk 4 * half + m of the 8 keys' rows;
-                        // the lane's register = dims 4tig .. 4tig+3 of key gid in that chunk
+                    for (int j = 0; j < KSTEPS / 2; ++j) {
+                        uint32_t r[4];
+                        ptx::ldsm_x4(sbase + stage_offset(key0 + (lm_mat & 1) * 8 + lm_row, 2 * j + (lm_mat >> 1)),
+                                     r[0], r[1], r[2], r[3]);
 #pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            uint32_t r[4];
-                            ptx::ldsm_x4(sbase + stage_offset(key0 + lm_row, 4 * half + lm_mat), r[0], r[1], r[2], r[3]);
-#pragma unroll
-                            for (int m = 0; m < 4; ++m) {
-                                const int ks = 4 * half + m;
-                                const uint32_t a[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
-                                ptx::mma_16816_f16(c, a, e4m3x2_to_f16x2(r[m]), e4m3x2_to_f16x2(r[m] >> 16));
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int ks = 0; ks < KSTEPS; ks += 2) {
-                            uint32_t b0, b1, b2, b3;
-                            ptx::ldsm_x4(sbase + stage_offset(key0 + lm_row, 2 * ks + lm_mat), b0, b1, b2, b3);
-                            const uint32_t a0[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
-                            const uint32_t a1[4] = {qa[ks + 1][0], 0u, qa[ks + 1][1], 0u};
-                            ptx::mma_16816_bf16(c, a0, b0, b1);
-                            ptx::mma_16816_bf16(c, a1, b2, b3);
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t lo = r[2 * h], hi = r[2 * h + 1];
+                            const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi),
+                                                   e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi >> 16)};
+                            ptx::mma_16816_f16(c[h], a, qb[2 * j + h][0], qb[2 * j + h][1]);
                         }
                     }
-                    if (row_real) {
-                        const int key = t * kSub + key0 + 2 * tig;
-                        s_sm[gid][key] = key < n ? c[0] * sl_row : -INFINITY;
-                        s_sm[gid][key + 1] = key + 1 < n ? c[1] * sl_row : -INFINITY;
+                } else {
+                    // matrices: (keys 0-7 | 8-15) x (dims 16ks .. +7 | 16ks+8 .. +15)
+#pragma unroll
+                    for (int ks = 0; ks < KSTEPS; ++ks) {
+                        uint32_t a[4];
+                        ptx::ldsm_x4(sbase + stage_offset(key0 + (lm_mat & 1) * 8 + lm_row, 2 * ks + (lm_mat >> 1)),
+                                     a[0], a[1], a[2], a[3]);
+                        ptx::mma_16816_bf16(c[ks & 1], a, qb[ks][0], qb[ks][1]);
                     }
+                }
+                // c[.][0..1]: key key0 + gid, heads 2tig / 2tig+1; c[.][2..3]: key key0 + gid + 8
+                const int ka = t * kSub + key0 + gid, kb8 = ka + 8;
+                if (hc0 < RG) {
+                    s_sm[hc0][ka] = ka < n ? (c[0][0] + c[1][0]) * sl0 : -INFINITY;
+                    s_sm[hc0][kb8] = kb8 < n ? (c[0][2] + c[1][2]) * sl0 : -INFINITY;
+                }
+                if (hc1 < RG) {
+                    s_sm[hc1][ka] = ka < n ? (c[0][1] + c[1][1]) * sl1 : -INFINITY;
+                    s_sm[hc1][kb8] = kb8 < n ? (c[0][3] + c[1][3]) * sl1 : -INFINITY;
                 }
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&empty[st]);
@@ -391,11 +454,12 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             }
             if (!gb.sync(sf)) break;
             // ------------------------------------------------------------ V pass
-            // bf16: acc[j] = column tile warp * NT + j (8 dims).  FP8: acc[2 * blk + par]
-            // holds the even (par 0) / odd (par 1) dims of 16-dim block 2 * warp + blk.
-            float acc[NT][4];
+            // warp w: O^T for head dims 16 VT w .. 16 VT (w+1) - 1, VT tiles of 16 (A = V^T).
+            // bf16: tile i rows = dims 16 (VT w + i) + (0..15).  FP8: tile i rows 0-7 = the
+            // even dims 16 (VT w + i) + 2r, rows 8-15 the odd dims 16 (VT w + i) + 2r + 1.
+            float acc[VT][4];
 #pragma unroll
-            for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+            for (int i = 0; i < VT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
             for (int t = 0; t * kSub < n; ++t) {
                 const uint32_t st = ring % C::kStages;
                 if (!wait_warp(&full[st], (ring / C::kStages) & 1u, sf)) { ok = false; break; }
@@ -416,43 +480,44 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                 const uint32_t sbase = ptx::smem_addr(stage);
 #pragma unroll
                 for (int kb = 0; kb < kSub; kb += 16) {
-                    // A operand: P of row gid for keys kb .. kb+15, zero beyond RG
-                    uint32_t pa[4] = {0u, 0u, 0u, 0u};
+                    // B operand: P^T, column gid = head gid, keys kb .. kb+15 (zero beyond RG)
+                    uint32_t pb0 = 0u, pb1 = 0u;
                     if (row_real) {
                         const float2 p0 = *reinterpret_cast<const float2 *>(&s_sm[gid][t * kSub + kb + 2 * tig]);
                         const float2 p1 = *reinterpret_cast<const float2 *>(&s_sm[gid][t * kSub + kb + 8 + 2 * tig]);
                         if constexpr (FP8) {
-                            pa[0] = ptx::pack_f16x2(p0.x, p0.y);
-                            pa[2] = ptx::pack_f16x2(p1.x, p1.y);
+                            pb0 = ptx::pack_f16x2(p0.x, p0.y);
+                            pb1 = ptx::pack_f16x2(p1.x, p1.y);
                         } else {
-                            pa[0] = pack2_bf16(p0.x, p0.y);
-                            pa[2] = pack2_bf16(p1.x, p1.y);
+                            pb0 = pack2_bf16(p0.x, p0.y);
+                            pb1 = pack2_bf16(p1.x, p1.y);
                         }
                     }
                     if constexpr (FP8) {
-                        // matrices: (keys kb..+7 | kb+8..+15) x (16-dim block 2 * warp | + 1);
-                        // a lane gets bytes {V[2tig][2gid], V[2tig][2gid+1], V[2tig+1][2gid],
-                        // V[2tig+1][2gid+1]} of its matrix
+                        // matrices: (keys kb..+7 | kb+8..+15) x (16-byte chunk 2w | 2w+1); a lane
+                        // gets bytes {V[2tig][2gid], V[2tig][2gid+1], V[2tig+1][2gid],
+                        // V[2tig+1][2gid+1]} of its matrix; one byte permute gives the key pair
+                        // of dim 2gid (low half) and of dim 2gid+1 (high half)
                         uint32_t r[4];
                         ptx::ldsm_x4_trans(sbase + stage_offset(kb + (lm_mat & 1) * 8 + lm_row, 2 * warp + (lm_mat >> 1)),
                                            r[0], r[1], r[2], r[3]);
 #pragma unroll
-                        for (int blk = 0; blk < 2; ++blk) {
-                            const uint32_t lo = __byte_perm(r[2 * blk], 0u, 0x3120);      // keys kb + 2tig, +1
-                            const uint32_t hi = __byte_perm(r[2 * blk + 1], 0u, 0x3120);  // keys kb + 8 + 2tig, +1
-                            ptx::mma_16816_f16(acc[2 * blk], pa, e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi));
-                            ptx::mma_16816_f16(acc[2 * blk + 1], pa, e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi >> 16));
+                        for (int i = 0; i < 2; ++i) {
+                            const uint32_t klo = __byte_perm(r[2 * i], 0u, 0x3120);      // keys kb + 2tig, +1
+                            const uint32_t khi = __byte_perm(r[2 * i + 1], 0u, 0x3120);  // keys kb + 8 + 2tig, +1
+                            const uint32_t a[4] = {e4m3x2_to_f16x2(klo), e4m3x2_to_f16x2(klo >> 16),
+                                                   e4m3x2_to_f16x2(khi), e4m3x2_to_f16x2(khi >> 16)};
+                            ptx::mma_16816_f16(acc[i], a, pb0, pb1);
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < NT; j += 2) {
-                            // matrices: (keys kb..+7 | kb+8..+15) x (column tile j | j+1)
-                            const int chunk = (warp * NT + j) + (lm_mat >> 1);
-                            const int row = kb + (lm_mat & 1) * 8 + lm_row;
-                            uint32_t b0, b1, b2, b3;
-                            ptx::ldsm_x4_trans(sbase + stage_offset(row, chunk), b0, b1, b2, b3);
-                            ptx::mma_16816_bf16(acc[j], pa, b0, b1);
-                            ptx::mma_16816_bf16(acc[j + 1], pa, b2, b3);
+                        for (int i = 0; i < VT; ++i) {
+                            // matrices: (dims of the tile 0-7 | 8-15) x (keys kb..+7 | kb+8..+15)
+                            const int chunk = 2 * (VT * warp + i) + (lm_mat & 1);
+                            const int row = kb + (lm_mat >> 1) * 8 + lm_row;
+                            uint32_t a[4];
+                            ptx::ldsm_x4_trans(sbase + stage_offset(row, chunk), a[0], a[1], a[2], a[3]);
+                            ptx::mma_16816_bf16(acc[i], a, pb0, pb1);
                         }
                     }
                 }
@@ -462,25 +527,28 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             }
             if (!ok) break;
             const int chunk = start / kChunk;
-            if (row_real) {
-                float *dst = p.part_o + (((size_t)b * p.Hq + h0 + gid) * p.S_max + chunk) * D;
-                if constexpr (FP8) {
-                    const float f = p.v_scale[g] / l_sm[gid];
+            // acc[i][0..1]: heads 2tig / 2tig+1 of tile row gid; acc[i][2..3]: of row gid + 8
+            {
+                const float f0 = hc0 < RG ? (FP8 ? p.v_scale[g] : 1.f) / l_sm[hc0] : 0.f;
+                const float f1 = hc1 < RG ? (FP8 ? p.v_scale[g] : 1.f) / l_sm[hc1] : 0.f;
+                float *dst0 = p.part_o + (((size_t)b * p.Hq + h0 + hc0) * p.S_max + chunk) * D;
+                float *dst1 = p.part_o + (((size_t)b * p.Hq + h0 + hc1) * p.S_max + chunk) * D;
 #pragma unroll
-                    for (int blk = 0; blk < 2; ++blk) {
-                        // acc[2blk] columns 2tig, 2tig+1 = dims 4tig, 4tig+2 of the block;
-                        // acc[2blk+1] the odd dims 4tig+1, 4tig+3
-                        const int col = (2 * warp + blk) * 16 + 4 * tig;
-                        *reinterpret_cast<float4 *>(dst + col) =
-                            make_float4(acc[2 * blk][0] * f, acc[2 * blk + 1][0] * f,
-                                        acc[2 * blk][1] * f, acc[2 * blk + 1][1] * f);
-                    }
-                } else {
-                    const float inv_l = 1.f / l_sm[gid];
-#pragma unroll
-                    for (int j = 0; j < NT; ++j) {
-                        const int col = (warp * NT + j) * 8 + 2 * tig;
-                        *reinterpret_cast<float2 *>(dst + col) = make_float2(acc[j][0] * inv_l, acc[j][1] * inv_l);
+                for (int i = 0; i < VT; ++i) {
+                    if constexpr (FP8) {
+                        const int dim = 16 * (VT * warp + i) + 2 * gid;  // rows gid / gid + 8 = dims +0 / +1
+                        if (hc0 < RG) *reinterpret_cast<float2 *>(dst0 + dim) = make_float2(acc[i][0] * f0, acc[i][2] * f0);
+                        if (hc1 < RG) *reinterpret_cast<float2 *>(dst1 + dim) = make_float2(acc[i][1] * f1, acc[i][3] * f1);
+                    } else {
+                        const int dim = 16 * (VT * warp + i) + gid;      // rows gid / gid + 8 = dims +0 / +8
+                        if (hc0 < RG) {
+                            dst0[dim] = acc[i][0] * f0;
+                            dst0[dim + 8] = acc[i][2] * f0;
+                        }
+                        if (hc1 < RG) {
+                            dst1[dim] = acc[i][1] * f1;
+                            dst1[dim + 8] = acc[i][3] * f1;
+                        }
                     }
                 }
             }
