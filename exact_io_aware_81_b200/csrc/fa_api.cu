@@ -406,8 +406,9 @@ struct CacheDesc {
 // contiguous cache length (ignored when paged: page_size * max_pages).
 int decode_general(const void *q, const CacheDesc &c, const int *seqlens, void *o, float *lse,
                    int B, int Hq, int Hkv, int Nmax, int d, float scale, void *workspace,
-                   size_t workspace_bytes, void *stream)
+                   size_t workspace_bytes, void *stream, int o_dtype = FA_BF16)
 {
+    if (o_dtype != FA_BF16 && o_dtype != FA_F32) return fail(FA_ERR_INVALID, "unknown output dtype %d", o_dtype);
     if (!q || !c.k || !c.v || !seqlens || !o) return fail(FA_ERR_INVALID, "null pointer argument");
     if (c.fp8 && (!c.k_scale || !c.v_scale)) return fail(FA_ERR_INVALID, "null scale pointer");
     if (c.paged && !c.block_table) return fail(FA_ERR_INVALID, "null block table");
@@ -469,7 +470,8 @@ int decode_general(const void *q, const CacheDesc &c, const int *seqlens, void *
     p.part_o = static_cast<float *>(workspace);
     p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
                                            align256((size_t)B * Hq * p.S_max * d * sizeof(float)));
-    p.o = static_cast<__nv_bfloat16 *>(o);
+    if (o_dtype == FA_F32) p.o_f32 = static_cast<float *>(o);
+    else p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
     p.B = B;
     p.Hq = Hq;
@@ -505,6 +507,43 @@ int fa_decode_paged(const void *q, const void *kpages, const void *vpages, const
 {
     const CacheDesc c{kpages, vpages, false, nullptr, nullptr, true, block_table, num_pages, page_size, max_pages};
     return decode_general(q, c, seqlens, o, lse, B, Hq, Hkv, 0, d, scale, workspace, workspace_bytes, stream);
+}
+
+int fa_decode_ex(const void *q, const void *kcache, const void *vcache, const int *seqlens, void *o,
+                 float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale, int o_dtype,
+                 void *workspace, size_t workspace_bytes, void *stream)
+{
+    const CacheDesc c{kcache, vcache, false, nullptr, nullptr, false, nullptr, 0, 0, 0};
+    return decode_general(q, c, seqlens, o, lse, B, Hq, Hkv, Nmax, d, scale, workspace, workspace_bytes,
+                          stream, o_dtype);
+}
+
+int fa_merge_lse(const float *o_parts, const float *lse_parts, int P, int rows, int d, void *o,
+                 float *lse, int o_dtype, void *stream)
+{
+    if (!o_parts || !lse_parts || !o) return fail(FA_ERR_INVALID, "null pointer argument");
+    if (P <= 0 || rows <= 0 || d <= 0) return fail(FA_ERR_INVALID, "sizes must be positive (P=%d rows=%d d=%d)", P, rows, d);
+    if (o_dtype != FA_BF16 && o_dtype != FA_F32) return fail(FA_ERR_INVALID, "unknown output dtype %d", o_dtype);
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    if ((long long)P * rows * d > 0x7fffffffffffLL) return fail(FA_ERR_UNSUPPORTED, "problem too large");
+    int dev, rc;
+    DeviceInfo *info;
+    if ((rc = current_device(&dev, &info)) != FA_OK) return rc;
+    fa::MergeLseParams m;
+    m.o_parts = o_parts;
+    m.lse_parts = lse_parts;
+    m.o = o_dtype == FA_BF16 ? static_cast<__nv_bfloat16 *>(o) : nullptr;
+    m.o_f32 = o_dtype == FA_F32 ? static_cast<float *>(o) : nullptr;
+    m.lse = lse;
+    m.P = P;
+    m.rows = rows;
+    const unsigned grid = (unsigned)((rows + fa::kMergeLseWarps - 1) / fa::kMergeLseWarps);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128) fa::fa_merge_lse_kernel<128><<<grid, 32 * fa::kMergeLseWarps, 0, st>>>(m);
+    else fa::fa_merge_lse_kernel<64><<<grid, 32 * fa::kMergeLseWarps, 0, st>>>(m);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
+    return ok();
 }
 
 int fa_decode_fp8(const void *q, const void *kcache, const void *vcache, const float *k_scale,

@@ -59,7 +59,8 @@ struct DecodeParams {
     const int *seqlens;       // (B)
     float *part_o;            // (B, Hq, S_max, D)  normalised partial outputs
     float *part_lse;          // (B, Hq, S_max)     partial log2-sum-exp (scaled scores)
-    __nv_bfloat16 *o;         // (B, Hq, D)
+    __nv_bfloat16 *o;         // (B, Hq, D) bf16 output, or
+    float *o_f32;             // (B, Hq, D) fp32 output when not null (o is then unused)
     float *lse;               // (B, Hq) natural log, may be null
     int B, Hq, Hkv, Nmax, R, S_max;
     int n_hg;      // head groups: Hq / RG
@@ -587,7 +588,10 @@ __global__ void __launch_bounds__(32 * kMergeWarps) fa_decode_merge_kernel(const
     const float *pl = p.part_lse + bh * p.S_max;
     const float *po = p.part_o + bh * p.S_max * D;
     if (S == 0) {
-        if (threadIdx.x < D) p.o[bh * D + threadIdx.x] = __float2bfloat16_rn(0.f);
+        if (threadIdx.x < D) {
+            if (p.o_f32) p.o_f32[bh * D + threadIdx.x] = 0.f;
+            else p.o[bh * D + threadIdx.x] = __float2bfloat16_rn(0.f);
+        }
         if (threadIdx.x == 0 && p.lse) p.lse[bh] = -INFINITY;
         return;
     }
@@ -618,9 +622,63 @@ __global__ void __launch_bounds__(32 * kMergeWarps) fa_decode_merge_kernel(const
             t += red[w][threadIdx.x];
             dsum += den_sm[w];
         }
-        p.o[bh * D + threadIdx.x] = __float2bfloat16_rn(t / dsum);
+        if (p.o_f32) p.o_f32[bh * D + threadIdx.x] = t / dsum;
+        else p.o[bh * D + threadIdx.x] = __float2bfloat16_rn(t / dsum);
         if (threadIdx.x == 0 && p.lse) p.lse[bh] = (M + ptx::lg2(dsum)) * kLn2;
     }
+}
+
+// Merge of P partial results computed elsewhere (for instance on other GPUs, each over
+// its own part of the keys): the log-sum-exp merge above with natural-log inputs.
+//   o_parts (P, rows, D) fp32, lse_parts (P, rows) natural log (-inf: no keys);
+//   o (rows, D) bf16 or o_f32 fp32; lse (rows) natural log, may be null.
+// One warp per row; lane owns D/32 consecutive elements.
+struct MergeLseParams {
+    const float *o_parts;
+    const float *lse_parts;
+    __nv_bfloat16 *o;
+    float *o_f32;
+    float *lse;
+    int P, rows;
+};
+
+constexpr int kMergeLseWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(32 * kMergeLseWarps) fa_merge_lse_kernel(const __grid_constant__ MergeLseParams m)
+{
+    constexpr int EPL = D / 32;
+    constexpr float kLog2e = 1.4426950408889634f;
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * kMergeLseWarps + (threadIdx.x >> 5);
+    if (row >= m.rows) return;
+    float M = -INFINITY;
+    for (int q = lane; q < m.P; q += 32) M = fmaxf(M, m.lse_parts[(size_t)q * m.rows + row]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float acc[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+    float den = 0.f;
+    if (M != -INFINITY) {
+        for (int q = 0; q < m.P; ++q) {
+            const float l = m.lse_parts[(size_t)q * m.rows + row];
+            if (l == -INFINITY) continue;  // a part with no keys: weight 0
+            const float w = ptx::ex2((l - M) * kLog2e);
+            den += w;
+            const float *src = m.o_parts + ((size_t)q * m.rows + row) * D + lane * EPL;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+        }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        const size_t i = (size_t)row * D + lane * EPL + e;
+        if (m.o_f32) m.o_f32[i] = acc[e] * inv;
+        else m.o[i] = __float2bfloat16_rn(acc[e] * inv);
+    }
+    if (lane == 0 && m.lse) m.lse[row] = den > 0.f ? M + logf(den) : -INFINITY;
 }
 
 }  // namespace fa

@@ -38,6 +38,8 @@ SIGNATURES = {
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "fa_decode_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
+    "fa_merge_lse": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P]),
     "fa_decode_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_paged_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                                  _P, _Z, _P]),
@@ -270,6 +272,70 @@ def _workspace(workspace, need, device):
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     return workspace
+
+
+def decode_ex(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens: torch.Tensor,
+              scale: Optional[float] = None, out_dtype: torch.dtype = torch.bfloat16,
+              workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+              lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
+    """fa_decode_ex: decode with a bf16 or fp32 output (fp32 keeps a partial result exact
+    enough to merge again with merge_lse)."""
+    _require(q, "q", torch.bfloat16, 3)
+    _require(kcache, "kcache", torch.bfloat16, 4)
+    _require(vcache, "vcache", torch.bfloat16, 4)
+    _require(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, d = q.shape
+    Bk, Hkv, Nmax, dk = kcache.shape
+    if (Bk, dk) != (B, d) or tuple(vcache.shape) != tuple(kcache.shape) or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, kcache, vcache and seqlens")
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    workspace = _workspace(workspace, decode_workspace_size(B, Hq, Nmax, d), q.device)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=out_dtype, device=q.device)
+    else:
+        _require(out, "out", out_dtype, 3)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _require(lse, "lse", torch.float32, 2)
+    rc = load().fa_decode_ex(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
+                             out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                             B, Hq, Hkv, Nmax, d, float(scale),
+                             FA_F32 if out_dtype == torch.float32 else FA_BF16, workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def merge_lse(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype: torch.dtype = torch.bfloat16,
+              out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None):
+    """fa_merge_lse: o_parts (P, *rows, d) fp32 and lse_parts (P, *rows) fp32 (natural log,
+    -inf = no keys) -> (o (*rows, d), lse (*rows))."""
+    _require(o_parts, "o_parts", torch.float32, o_parts.dim())
+    _require(lse_parts, "lse_parts", torch.float32, lse_parts.dim())
+    if o_parts.dim() < 3 or tuple(o_parts.shape[:-1]) != tuple(lse_parts.shape):
+        raise ValueError("o_parts must be (P, *rows, d) and lse_parts (P, *rows)")
+    P, d = o_parts.shape[0], o_parts.shape[-1]
+    row_shape = tuple(o_parts.shape[1:-1])
+    rows = 1
+    for x in row_shape:
+        rows *= x
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    if out is None:
+        out = torch.empty(row_shape + (d,), dtype=out_dtype, device=o_parts.device)
+    else:
+        _require(out, "out", out_dtype, len(row_shape) + 1)
+    if lse is None:
+        lse = torch.empty(row_shape, dtype=torch.float32, device=o_parts.device)
+    rc = load().fa_merge_lse(o_parts.data_ptr(), lse_parts.data_ptr(), P, rows, d, out.data_ptr(),
+                             lse.data_ptr(), FA_F32 if out_dtype == torch.float32 else FA_BF16,
+                             _stream_handle(stream))
+    _check(rc)
+    return out, lse
 
 
 def decode_fp8(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, k_scale: torch.Tensor,

@@ -115,6 +115,33 @@ FA_API int fa_decode(const void *q, const void *kcache, const void *vcache, cons
               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * As fa_decode, with the output element type chosen by o_dtype: FA_BF16 or FA_F32 (o is
+ * then (B, Hq, d) fp32).  The fp32 output keeps partial results exact enough to be merged
+ * again, as fa_merge_lse does for a cache split across devices.
+ */
+FA_API int fa_decode_ex(const void *q, const void *kcache, const void *vcache, const int *seqlens,
+                 void *o, float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale,
+                 int o_dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Log-sum-exp merge of P partial attention results over disjoint key sets (the same
+ * rescaling the online softmax applies between key blocks, youngju.dev "attention
+ * variants" section 3, applied across parts): for every row,
+ *     M = max_p lse_p,  w_p = exp(lse_p - M),  o = sum_p w_p o_p / sum_p w_p,
+ *     lse = M + ln sum_p w_p.
+ * Used for context-parallel decode: each device decodes its own slab of every sequence's
+ * keys (fa_decode_ex with FA_F32), the (o, lse) pairs are all-gathered, and this call
+ * combines them into the result over the whole cache.
+ *   o_parts   (P, rows, d) fp32 device memory;  lse_parts (P, rows) fp32, natural log,
+ *             -inf for a part that saw no key (its o_p is ignored).
+ *   o         (rows, d) written, bf16 or fp32 (o_dtype);  lse (rows) written, or NULL.
+ *   A row whose every part is -inf gets o = 0 and lse = -inf.  d in {64, 128}.
+ * This library adds it: the pages merge only the blocks of one pass.
+ */
+FA_API int fa_merge_lse(const float *o_parts, const float *lse_parts, int P, int rows, int d,
+                 void *o, float *lse, int o_dtype, void *stream);
+
+/*
  * Decode step over a paged KV cache (youngju.dev "attention variants", section 5: the
  * cache is cut into fixed-size blocks managed like virtual-memory pages, which removes
  * fragmentation).  The page layout is this library's choice:

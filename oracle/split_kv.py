@@ -10,11 +10,31 @@ applied across independently computed chunks of the cache:
           o = sum_s w_s o_s / sum_s w_s,   lse = M + ln sum_s w_s
 
 Written in float64 numpy, one (b, h) at a time; only for checking that every chunk size
-reproduces the unsplit definition.
+reproduces the unsplit definition.  ``merge_lse`` is the merge step alone, over any number
+of partials (the cross-device merge of context-parallel decode uses the same algebra).
 """
 from __future__ import annotations
 
 import numpy as np
+
+
+def merge_lse(o_parts, lse_parts):
+    """Merge P partial results: o_parts (P, ..., d), lse_parts (P, ...) natural-log sums.
+
+    A partial with lse = -inf (no keys) has weight 0; if every partial has none, o = 0 and
+    lse = -inf.  Returns (o (..., d), lse (...)) in float64.
+    """
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    M = lse_parts.max(axis=0)
+    empty = np.isneginf(M)
+    Ms = np.where(empty, 0.0, M)
+    w = np.exp(lse_parts - Ms)                      # exp(-inf) = 0 for empty partials
+    den = w.sum(axis=0)
+    num = (w[..., None] * np.where(np.isneginf(lse_parts)[..., None], 0.0, o_parts)).sum(axis=0)
+    o = np.where(empty[..., None], 0.0, num / np.where(empty, 1.0, den)[..., None])
+    lse = np.where(empty, -np.inf, Ms + np.log(np.where(empty, 1.0, den)))
+    return o, lse
 
 
 def split_kv_decode(q, kcache, vcache, seqlens, scale, chunk):
@@ -41,9 +61,6 @@ def split_kv_decode(q, kcache, vcache, seqlens, scale, chunk):
                 parts.append(((e @ vv) / e.sum(), m + np.log(e.sum())))
             if not parts:
                 continue
-            lses = np.array([p[1] for p in parts])
-            M = lses.max()
-            w = np.exp(lses - M)
-            o[b, h] = sum(wi * p[0] for wi, p in zip(w, parts)) / w.sum()
-            lse[b, h] = M + np.log(w.sum())
+            o[b, h], lse[b, h] = merge_lse(np.stack([p[0] for p in parts]),
+                                           np.array([p[1] for p in parts]))
     return o, lse

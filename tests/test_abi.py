@@ -209,3 +209,24 @@ def test_decode_paged_fp8_rejects(lib):
     rc = lib.fa_decode_paged_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 10,
                                  40, 5, 128, 0.1, FAKE, 1 << 20, None)
     assert rc == ops.FA_ERR_UNSUPPORTED              # page size not a multiple of 16
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(op=None), ops.FA_ERR_INVALID),
+    (dict(P=0), ops.FA_ERR_INVALID),
+    (dict(rows=0), ops.FA_ERR_INVALID),
+    (dict(dt=3), ops.FA_ERR_INVALID),
+    (dict(d=96), ops.FA_ERR_UNSUPPORTED),
+])
+def test_merge_lse_rejects(lib, kw, status):
+    a = dict(op=FAKE, lp=FAKE, P=2, rows=4, d=128, o=FAKE, lse=None, dt=0)
+    a.update(kw)
+    assert lib.fa_merge_lse(a["op"], a["lp"], a["P"], a["rows"], a["d"], a["o"], a["lse"], a["dt"], None) == status
+
+
+def test_decode_ex_rejects(lib):
+    ws = lib.fa_decode_workspace_size(2, 8, 300, 128)
+    rc = lib.fa_decode_ex(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 300, 128, 0.1, 7, FAKE, ws, None)
+    assert rc == ops.FA_ERR_INVALID                  # unknown output dtype
+    rc = lib.fa_decode_ex(FAKE, FAKE, FAKE, None, FAKE, None, 2, 8, 2, 300, 128, 0.1, 1, FAKE, ws, None)
+    assert rc == ops.FA_ERR_INVALID                  # no seqlens

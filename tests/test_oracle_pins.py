@@ -416,6 +416,30 @@ def pin_fp8_decode_library_sdpa():
         assert torch.allclose(lse[b], rl[0, :, 0], atol=1e-12, rtol=0)
 
 
+def pin_context_parallel_merge_equals_unsplit():
+    """The cache cut into R contiguous shards (some empty for short sequences), each decoded
+    on its own by the C oracle and merged by merge_lse, equals the unsplit decode."""
+    from oracle.split_kv import merge_lse
+    B, Hq, Hkv, Nmax, d = 4, 8, 2, 400, 32
+    w = inputs.make_decode(B, Hq, Hkv, Nmax, d, seed=90, len_range=(0, Nmax))
+    sl = torch.tensor([0, 57, 400, 250], dtype=torch.int32)
+    full_o, full_l = oracle.decode(w.q, w.kcache, w.vcache, sl, w.scale)
+    for R in (1, 2, 3, 4):
+        C = -(-Nmax // R)
+        parts_o, parts_l = [], []
+        for r in range(R):
+            kc = w.kcache[:, :, r * C:(r + 1) * C].contiguous()
+            vc = w.vcache[:, :, r * C:(r + 1) * C].contiguous()
+            slr = (sl - r * C).clamp(0, kc.shape[2]).to(torch.int32)
+            o, l = oracle.decode(w.q, kc, vc, slr, w.scale)
+            parts_o.append(o.numpy()); parts_l.append(l.numpy())
+        mo, ml = merge_lse(np.stack(parts_o), np.stack(parts_l))
+        assert np.allclose(mo, full_o.numpy(), atol=1e-12, rtol=0), R
+        fin = np.isfinite(full_l.numpy())
+        assert np.allclose(ml[fin], full_l.numpy()[fin], atol=1e-12, rtol=0)
+        assert np.isneginf(ml[~fin]).all() and (mo[0] == 0).all()
+
+
 PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]
 
 
