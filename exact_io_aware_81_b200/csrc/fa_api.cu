@@ -193,7 +193,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     if ((rc = encode_rows_map(&p.tm_q, q, d, Nq, (long long)B * Hq)) != FA_OK) return rc;
     if ((rc = encode_rows_map(&p.tm_k, k, d, Nk, (long long)B * Hkv)) != FA_OK) return rc;
     if ((rc = encode_rows_map(&p.tm_v, v, d, Nk, (long long)B * Hkv)) != FA_OK) return rc;
-    if (o_dtype == FA_BF16 && (rc = encode_rows_map(&p.tm_o, o, d, Nq, (long long)B * Hq)) != FA_OK) return rc;
+    if (o_dtype == FA_BF16 && (rc = encode_rows_map(&p.tm_o, o, d, Nq, (long long)B * Hq, 32)) != FA_OK) return rc;
     p.o = o;
     p.lse = lse;
     p.B = B;

@@ -47,7 +47,7 @@ struct PrefillParams {
     CUtensorMap tm_q;  // (d, Nq, B*Hq) bf16, box (64, 128, 1), 128B swizzle
     CUtensorMap tm_k;  // (d, Nk, B*Hkv)
     CUtensorMap tm_v;  // (d, Nk, B*Hkv)
-    CUtensorMap tm_o;  // (d, Nq, B*Hq) bf16 output, box (64, 128, 1), 128B swizzle
+    CUtensorMap tm_o;  // (d, Nq, B*Hq) bf16 output, box (64, 32, 1), 128B swizzle: one warp's rows
     void *o;
     float *lse;
     int B, Hq, Hkv, Nq, Nk;
@@ -88,8 +88,8 @@ struct Cfg {
     static constexpr int kKVOff = 4 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
     // barriers: kv_full[S], kv_empty[S], q_full[2 sets][2], q_empty[2 sets][2], s_full[2],
-    //           p_ready[2], o_done[2], o_free[2], teardown, epilogue group[2], p_half[2]
-    static constexpr int kNumBars = 2 * kStages + 21;
+    //           p_ready[2], o_done[2], o_free[2], teardown, p_half[2]
+    static constexpr int kNumBars = 2 * kStages + 19;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 };
@@ -323,8 +323,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
     uint64_t *o_done = q_full + 12;
     uint64_t *o_free = q_full + 14;
     uint64_t *teardown = q_full + 16;
-    uint64_t *epi_group = q_full + 17;  // [2]: the four warps of a softmax warpgroup
-    uint64_t *p_half = q_full + 19;     // [2]: first 64 keys of P_s written
+    uint64_t *p_half = q_full + 17;     // [2]: first 64 keys of P_s written
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
     int *stop_flag = reinterpret_cast<int *>(smem + C::kMiscOff + 4);
 
@@ -340,9 +339,10 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             ptx::mbar_init(&q_full[s], 1);
             ptx::mbar_init(&q_full[2 + s], 1);
             // a Q slot is free again once its last S MMA is done (MMA commit) and the
-            // epilogue, which stages O through the same slot, has stored it (one arrive)
-            ptx::mbar_init(&q_empty[s], 2);
-            ptx::mbar_init(&q_empty[2 + s], 2);
+            // epilogue, which stages O through the same slot, has stored it (one arrive
+            // per warp of the softmax warpgroup)
+            ptx::mbar_init(&q_empty[s], 5);
+            ptx::mbar_init(&q_empty[2 + s], 5);
             ptx::mbar_init(&s_full[s], 1);
             ptx::mbar_init(&p_ready[s], 128);
             ptx::mbar_init(&p_half[s], 128);
@@ -350,8 +350,6 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             ptx::mbar_init(&o_free[s], 128);
         }
         ptx::mbar_init(teardown, 1);
-        ptx::mbar_init(&epi_group[0], 4);
-        ptx::mbar_init(&epi_group[1], 4);
         *stop_flag = 0;
         ptx::fence_barrier_init();
     }
@@ -585,7 +583,6 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         const uint32_t tS = tmem + lane_base + 128u * s;        // S_s, and P_s over it
         const uint32_t tO = tmem + lane_base + 256u + 128u * s;  // O_s
         const float sl2 = p.scale_log2;
-        GroupBarrier eg{&epi_group[s], 0u};
         uint32_t s_ph = 0, units = 0;
         Unit w;
         for (int u = next_unit<WINDOW>(p, 2 * (int)blockIdx.x, w); u >= 0; u = next_unit<WINDOW>(p, unit_step(u), w)) {
@@ -679,8 +676,9 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             // ------------------------------------------------------------- epilogue
             // O_s / lo leaves TMEM as soon as it is read (o_free lets the next unit's first
             // P V overwrite it).  bf16 output is staged, 128-byte swizzled, in this unit's Q
-            // slot -- no MMA reads it any more -- and written by one TMA store; the slot is
-            // then handed back to the producer.  fp32 output is stored row by row.
+            // slot -- no MMA reads it any more -- and each warp writes its own 32 rows with
+            // one TMA store, then hands its part of the slot back to the producer, so no
+            // warp waits for another.  fp32 output is stored row by row.
             if (!wait_warp(&o_done[s], units & 1u, sf)) break;
             ptx::tc_fence_after();
             const bool valid = row < p.Nq;
@@ -703,7 +701,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                                              __uint_as_float(ov[4 * e + 2]) * inv_l,
                                              __uint_as_float(ov[4 * e + 3]) * inv_l);
                 }
-                if (tid == 0) ptx::mbar_arrive(&q_empty[qi]);
+                if (lane == 0) ptx::mbar_arrive(&q_empty[qi]);
             } else {
                 uint8_t *stage = smem + C::kQOff + qi * C::kTileBytes;
 #pragma unroll
@@ -718,20 +716,24 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     *reinterpret_cast<uint4 *>(stage + slab * kChunkBytes + tid * 128 + chunk * 16) = v4;
                 }
                 ptx::fence_proxy_async_smem();
-                if (!eg.sync(sf)) break;
-                if (tid == 0) {
+                __syncwarp();
+                if (lane == 0) {
+                    const int wr = 32 * (warp & 3);  // this warp's rows of the tile
+                    if (r0 + wr < p.Nq) {            // (rows past Nq are never stored)
 #pragma unroll
-                    for (int c = 0; c < D / 64; ++c)
-                        ptx::tma_store_3d(&p.tm_o, stage + c * kChunkBytes, 64 * c, r0, w.b * p.Hq + h);
-                    ptx::bulk_commit_group();
-                    ptx::bulk_wait_group_read0();
+                        for (int c = 0; c < D / 64; ++c)
+                            ptx::tma_store_3d(&p.tm_o, stage + c * kChunkBytes + wr * 128, 64 * c, r0 + wr,
+                                              w.b * p.Hq + h);
+                        ptx::bulk_commit_group();
+                        ptx::bulk_wait_group_read0();
+                    }
                     ptx::mbar_arrive(&q_empty[qi]);
                 }
             }
             if (valid) p.lse[orow] = (m + ptx::lg2(l)) * kLn2;
             ++units;
         }
-        if (!OUT_F32 && tid == 0) ptx::bulk_wait_group0();  // stores complete before exit
+        if (!OUT_F32 && lane == 0) ptx::bulk_wait_group0();  // stores complete before exit
     }
 
     else {
