@@ -27,24 +27,25 @@
 // pages; the consumers and the merge are unchanged.
 //
 // FP8 caches (E4M3 bytes with one dequantization scale per K/V head for K and one for V;
-// youngju.dev sections 5 and 7 name FP8 KV caches) halve the bytes read.  Each E4M3 pair
-// is converted exactly to fp16 in registers and the same mma.sync tiles run on fp16
-// operands:
+// youngju.dev sections 5 and 7 name FP8 KV caches) halve the bytes read.  Each E4M3 value
+// becomes an fp16 value in registers by moving its bit fields (sign to bit 15, exponent and
+// mantissa to bits 7-13): that fp16 value is the E4M3 value times 2^-8 exactly, subnormals
+// included, because the two exponent biases differ by 8.  The conversion pairs bytes 0 and
+// 2, and 1 and 3, of a 32-bit register, and the same mma.sync tiles run on fp16 operands:
 //   K pass: ldmatrix (not transposed) hands a lane 4 consecutive dims of one key; the
-//     MMA's contraction index is permuted so that those 4 dims are the lane's two B
-//     registers, and q is loaded in the same permuted order (so no transpose is needed).
-//     q is scaled per row by an exact power of two 2^e so that its largest element lies
-//     in [2^14, 2^15) before the fp16 conversion (every bf16 value in that range is an
-//     fp16 value); the factor k_scale * 2^-e is applied to the fp32 scores.
-//   V pass: a transposing 16-bit ldmatrix hands a lane 2 dims x 2 keys; one byte permute
-//     splits them into the key pairs of an even and an odd dim, which are the B
-//     registers of two MMAs whose output columns are the even and the odd dims.  P is
-//     converted to fp16 and v_scale is applied with the final 1 / l.
+//     MMA's contraction index is permuted so that dims (0, 2) and (1, 3) of those 4 are
+//     the lane's A registers, and q is loaded in the same permuted order (so no transpose
+//     is needed).  q is scaled per row by an exact power of two 2^e so that its largest
+//     element lies in [2^14, 2^15) before the fp16 conversion (every bf16 value in that
+//     range is an fp16 value); k_scale * 2^8 * 2^-e is applied to the fp32 scores.
+//   V pass: a transposing 16-bit ldmatrix hands a lane 2 dims x 2 keys as bytes
+//     {key 0 dim 0, key 0 dim 1, key 1 dim 0, key 1 dim 1}: bytes (0, 2) are the key pair
+//     of the even dim and (1, 3) that of the odd dim, the A rows of the even and the odd
+//     output dims.  P is converted to fp16 and v_scale * 2^8 is applied with the final 1 / l.
 #pragma once
 
 #include <cstdint>
 #include <cuda_bf16.h>
-#include <cuda_fp8.h>
 
 #include "fa_common.cuh"
 #include "ptx_sm100.cuh"
@@ -115,12 +116,12 @@ __device__ __forceinline__ uint32_t stage_offset(int r, int c)
 
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) { return ptx::pack_bf16x2(lo, hi); }
 
-// Two E4M3 bytes (low byte -> low half) to packed fp16; exact for every finite E4M3 value.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes)
-{
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_bytes & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
+// E4M3 bytes 0 and 2 (even) / 1 and 3 (odd) of x to packed fp16 times 2^-8, exactly: the
+// sign moves to bit 15 and exponent + mantissa to bits 7-13 of each half
+__device__ __forceinline__ uint32_t e4m3_even_f16x2(uint32_t x) { return ((x << 8) & 0x80008000u) | ((x << 7) & 0x3F803F80u); }
+__device__ __forceinline__ uint32_t e4m3_odd_f16x2(uint32_t x) { return (x & 0x80008000u) | ((x >> 1) & 0x3F803F80u); }
+
+
 
 }  // namespace decode
 
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             // or head dims (V pass) in M = 16, so no MMA row is padding.
             // B operand of S^T = K Q^T: column gid = query head h0 + gid (zero beyond RG).
             // bf16: K step ks holds dims 16ks + 2tig + {0,1} and 16ks + 8 + 2tig + {0,1}.
-            // FP8:  K step ks holds dims 16ks + 4tig + {0,1} and 16ks + 4tig + {2,3} (the
+            // FP8:  K step ks holds dims 16ks + 4tig + {0,2} and 16ks + 4tig + {1,3} (the
             //       permuted contraction order of the K pass), as fp16 scaled by 2^e.
             uint32_t qb[KSTEPS][2];
             // factors from the MMA result to log2-domain scores of heads 2tig and 2tig+1
@@ -367,10 +368,10 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                     const float down = __uint_as_float((uint32_t)(127 - e) << 23);
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks) {
-                        qb[ks][0] = ptx::pack_f16x2(qv[ks][0] * up, qv[ks][1] * up);
-                        qb[ks][1] = ptx::pack_f16x2(qv[ks][2] * up, qv[ks][3] * up);
+                        qb[ks][0] = ptx::pack_f16x2(qv[ks][0] * up, qv[ks][2] * up);
+                        qb[ks][1] = ptx::pack_f16x2(qv[ks][1] * up, qv[ks][3] * up);
                     }
-                    const float sl_own = p.scale_log2 * p.k_scale[g] * down;  // head gid
+                    const float sl_own = p.scale_log2 * p.k_scale[g] * 256.f * down;  // head gid
                     sl0 = __shfl_sync(0xffffffffu, sl_own, 8 * tig);          // head 2tig
                     sl1 = __shfl_sync(0xffffffffu, sl_own, 8 * tig + 4);      // head 2tig+1
                 } else {
@@ -404,8 +405,8 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             const uint32_t lo = r[2 * h], hi = r[2 * h + 1];
-                            const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi),
-                                                   e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi >> 16)};
+                            const uint32_t a[4] = {e4m3_even_f16x2(lo), e4m3_even_f16x2(hi),
+                                                   e4m3_odd_f16x2(lo), e4m3_odd_f16x2(hi)};
                             ptx::mma_16816_f16(c[h], a, qb[2 * j + h][0], qb[2 * j + h][1]);
                         }
                     }
@@ -497,17 +498,16 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                     if constexpr (FP8) {
                         // matrices: (keys kb..+7 | kb+8..+15) x (16-byte chunk 2w | 2w+1); a lane
                         // gets bytes {V[2tig][2gid], V[2tig][2gid+1], V[2tig+1][2gid],
-                        // V[2tig+1][2gid+1]} of its matrix; one byte permute gives the key pair
-                        // of dim 2gid (low half) and of dim 2gid+1 (high half)
+                        // V[2tig+1][2gid+1]} of its matrix: bytes (0, 2) are the key pair of
+                        // dim 2gid, bytes (1, 3) that of dim 2gid+1
                         uint32_t r[4];
                         ptx::ldsm_x4_trans(sbase + stage_offset(kb + (lm_mat & 1) * 8 + lm_row, 2 * warp + (lm_mat >> 1)),
                                            r[0], r[1], r[2], r[3]);
 #pragma unroll
                         for (int i = 0; i < 2; ++i) {
-                            const uint32_t klo = __byte_perm(r[2 * i], 0u, 0x3120);      // keys kb + 2tig, +1
-                            const uint32_t khi = __byte_perm(r[2 * i + 1], 0u, 0x3120);  // keys kb + 8 + 2tig, +1
-                            const uint32_t a[4] = {e4m3x2_to_f16x2(klo), e4m3x2_to_f16x2(klo >> 16),
-                                                   e4m3x2_to_f16x2(khi), e4m3x2_to_f16x2(khi >> 16)};
+                            const uint32_t klo = r[2 * i], khi = r[2 * i + 1];
+                            const uint32_t a[4] = {e4m3_even_f16x2(klo), e4m3_odd_f16x2(klo),
+                                                   e4m3_even_f16x2(khi), e4m3_odd_f16x2(khi)};
                             ptx::mma_16816_f16(acc[i], a, pb0, pb1);
                         }
                     } else {
@@ -530,8 +530,8 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             const int chunk = start / kChunk;
             // acc[i][0..1]: heads 2tig / 2tig+1 of tile row gid; acc[i][2..3]: of row gid + 8
             {
-                const float f0 = hc0 < RG ? (FP8 ? p.v_scale[g] : 1.f) / l_sm[hc0] : 0.f;
-                const float f1 = hc1 < RG ? (FP8 ? p.v_scale[g] : 1.f) / l_sm[hc1] : 0.f;
+                const float f0 = hc0 < RG ? (FP8 ? 256.f * p.v_scale[g] : 1.f) / l_sm[hc0] : 0.f;
+                const float f1 = hc1 < RG ? (FP8 ? 256.f * p.v_scale[g] : 1.f) / l_sm[hc1] : 0.f;
                 float *dst0 = p.part_o + (((size_t)b * p.Hq + h0 + hc0) * p.S_max + chunk) * D;
                 float *dst1 = p.part_o + (((size_t)b * p.Hq + h0 + hc1) * p.S_max + chunk) * D;
 #pragma unroll
