@@ -205,6 +205,16 @@ def oracle_prefill_rate(w, target_s: float, seed: int = 0):
 
 # ------------------------------------------------------------------ reference arm
 
+def step_config(world):
+    """The workload of one step, shared by both arms."""
+    return {
+        "workload": f"{inputs.WORKLOADS[2]} + {inputs.WORKLOADS[5]}",
+        "global_batch": 8 * world, "seq_len": 2048, "decode_batch": 32 * world,
+        "parallelism": f"replicas: dp{world} (independent problems per GPU, no collective)",
+        "l2": "inputs larger than L2 (prefill 537 MB, decode caches 1074 MB)",
+    }
+
+
 def run_reference(args, rank, world):
     out = None
     if rank == 0:
@@ -225,15 +235,15 @@ def run_reference(args, rank, world):
                 times.append(dt)
                 flops.append(4.0 * d * B * Hq * per)
         value = sum(flops) / sum(times) / 1e12
-        sample = f"{nrows} sampled query rows per (b, h) of the prefill workload per step, all 256 (b, h)"
+        sample = (f"{nrows} sampled query rows per (b, h) of the prefill workload per step, all 256 (b, h); "
+                  "the value is the prefill throughput, as in the other arm (rank 0 only)")
         out = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": inputs.WORKLOADS[2], "global_batch": 8, "seq_len": 2048,
-                       "parallelism": "replicas only (rank 0 runs the CPU oracle)"},
+            "config": step_config(world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -386,12 +396,7 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": f"{inputs.WORKLOADS[2]} + {inputs.WORKLOADS[5]}",
-            "global_batch": 8 * world, "seq_len": 2048, "decode_batch": 32 * world,
-            "parallelism": f"replicas: dp{world} (independent problems per GPU, no collective)",
-            "l2": "inputs larger than L2 (prefill 537 MB, decode caches 1074 MB)",
-        },
+        "config": step_config(world),
         "roofline": {
             "bound": "tensor", "achieved": pre_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
             "frac": pre_tflops / tensor_peak, "traffic": pre_traffic,
