@@ -328,11 +328,48 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
         const int lm_mat = lane >> 3;
         const int n_items = count_items(p);
         ItemCursor cur;
+        // The q rows of an item (the B operand of the K pass; for FP8 also its k_scale) are
+        // loaded one item ahead, so that their latency overlaps the previous item's passes.
+        // bf16: r[2ks], r[2ks+1] = dims 16ks + 2tig + {0,1}, 16ks + 8 + 2tig + {0,1};
+        // FP8: r[2ks], r[2ks+1] = dims 16ks + 4tig + {0,1}, 16ks + 4tig + {2,3}.
+        auto load_q = [&](int qb_, int qhg, uint32_t (&r)[2 * KSTEPS], float &ksc) {
+            const __nv_bfloat16 *qrow = p.q + ((size_t)qb_ * p.Hq + qhg * RG + (row_real ? gid : 0)) * D;
+            if constexpr (FP8) {
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    const uint2 raw = row_real ? *reinterpret_cast<const uint2 *>(qrow + 16 * ks + 4 * tig)
+                                               : make_uint2(0u, 0u);
+                    r[2 * ks] = raw.x;
+                    r[2 * ks + 1] = raw.y;
+                }
+                ksc = p.k_scale[qhg * RG / p.R];
+            } else {
+                const uint32_t *qw = reinterpret_cast<const uint32_t *>(qrow);
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    r[2 * ks] = row_real ? qw[8 * ks + tig] : 0u;
+                    r[2 * ks + 1] = row_real ? qw[8 * ks + 4 + tig] : 0u;
+                }
+            }
+        };
+        int b = 0, hg = 0, start = 0, n = 0;
+        uint32_t qraw[2 * KSTEPS];
+        float kscale = 0.f;
+        if ((int)blockIdx.x < n_items) {
+            decode_item(p, cur, blockIdx.x, b, hg, start, n);
+            load_q(b, hg, qraw, kscale);
+        }
         for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-            int b, hg, start, n;
-            decode_item(p, cur, it, b, hg, start, n);
             const int h0 = hg * RG;
             const int g = h0 / p.R;
+            const int nit = it + gridDim.x;
+            int nb = 0, nhg = 0, nstart = 0, nn = 0;
+            uint32_t qnext[2 * KSTEPS];
+            float knext = 0.f;
+            if (nit < n_items) {
+                decode_item(p, cur, nit, nb, nhg, nstart, nn);
+                load_q(nb, nhg, qnext, knext);
+            }
             // The MMAs put the query heads in the N = 8 dimension (RG <= 8) and keys (K pass)
             // or head dims (V pass) in M = 16, so no MMA row is padding.
             // B operand of S^T = K Q^T: column gid = query head h0 + gid (zero beyond RG).
@@ -343,18 +380,15 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             // factors from the MMA result to log2-domain scores of heads 2tig and 2tig+1
             float sl0 = p.scale_log2, sl1 = p.scale_log2;
             {
-                const __nv_bfloat16 *qrow = p.q + ((size_t)b * p.Hq + h0 + (row_real ? gid : 0)) * D;
                 if constexpr (FP8) {
                     float qv[KSTEPS][4];
                     float amax = 0.f;
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks) {
-                        const uint2 raw = row_real ? *reinterpret_cast<const uint2 *>(qrow + 16 * ks + 4 * tig)
-                                                   : make_uint2(0u, 0u);
-                        qv[ks][0] = __uint_as_float(raw.x << 16);
-                        qv[ks][1] = __uint_as_float(raw.x & 0xffff0000u);
-                        qv[ks][2] = __uint_as_float(raw.y << 16);
-                        qv[ks][3] = __uint_as_float(raw.y & 0xffff0000u);
+                        qv[ks][0] = __uint_as_float(qraw[2 * ks] << 16);
+                        qv[ks][1] = __uint_as_float(qraw[2 * ks] & 0xffff0000u);
+                        qv[ks][2] = __uint_as_float(qraw[2 * ks + 1] << 16);
+                        qv[ks][3] = __uint_as_float(qraw[2 * ks + 1] & 0xffff0000u);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qv[ks][e]));
                     }
@@ -371,15 +405,14 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                         qb[ks][0] = ptx::pack_f16x2(qv[ks][0] * up, qv[ks][2] * up);
                         qb[ks][1] = ptx::pack_f16x2(qv[ks][1] * up, qv[ks][3] * up);
                     }
-                    const float sl_own = p.scale_log2 * p.k_scale[g] * 256.f * down;  // head gid
+                    const float sl_own = p.scale_log2 * kscale * 256.f * down;  // head gid
                     sl0 = __shfl_sync(0xffffffffu, sl_own, 8 * tig);          // head 2tig
                     sl1 = __shfl_sync(0xffffffffu, sl_own, 8 * tig + 4);      // head 2tig+1
                 } else {
-                    const uint32_t *qw = reinterpret_cast<const uint32_t *>(qrow);
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks) {
-                        qb[ks][0] = row_real ? qw[8 * ks + tig] : 0u;
-                        qb[ks][1] = row_real ? qw[8 * ks + 4 + tig] : 0u;
+                        qb[ks][0] = qraw[2 * ks];
+                        qb[ks][1] = qraw[2 * ks + 1];
                     }
                 }
             }
@@ -558,6 +591,13 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                     m_sm[threadIdx.x] + ptx::lg2(l_sm[threadIdx.x]);
             // scores and m/l are rewritten by the next item
             if (!gb.sync(sf)) break;
+            b = nb;
+            hg = nhg;
+            start = nstart;
+            n = nn;
+            kscale = knext;
+#pragma unroll
+            for (int i = 0; i < 2 * KSTEPS; ++i) qraw[i] = qnext[i];
         }
     }
     __syncthreads();
