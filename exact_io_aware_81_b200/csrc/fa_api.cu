@@ -236,6 +236,10 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
 
 long long decode_splits(int Nmax) { return (Nmax + fa::decode::kChunk - 1) / fa::decode::kChunk; }
 
+// Rows per TMA box of the decode kernels: the 64-row stages of the bf16 kernel and the
+// 64-key blocks of the FP8 one.
+int decode_block_keys(int, bool fp8) { return fp8 ? fa::decode::kSK : fa::decode::kSub; }
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t decode_ws_bytes(int B, int Hq, int Nmax, int d)
@@ -245,18 +249,22 @@ size_t decode_ws_bytes(int B, int Hq, int Nmax, int d)
     return align256((size_t)B * Hq * S * d * sizeof(float)) + align256((size_t)B * Hq * S * sizeof(float));
 }
 
-// Persistent split kernel: one CTA per SM (at most one per work item).
+// Persistent split kernel, 3 CTAs per SM (at most one per candidate work item): the bf16
+// kernel, or the FP8 one (head dim 128).
 template <int D, int RG, bool PAGED, bool FP8>
 int launch_split(fa::DecodeParams p, DeviceInfo *info, cudaStream_t st)
 {
-    using C = fa::decode::SplitCfg<D, RG, FP8>;
-    static_assert(C::kSmemBytes * fa::decode::kCtasPerSm <= 227 * 1024, "decode CTAs per SM do not fit");
+    static_assert(!FP8 || D == 128, "FP8 caches: head dim 128");
+    constexpr int smem = FP8 ? fa::decode::WorkerCfg<RG>::kSmemBytes : fa::decode::SplitCfg<D, RG>::kSmemBytes;
+    static_assert(smem * fa::decode::kCtasPerSm <= 227 * 1024, "decode CTAs per SM do not fit");
+    void (*kern)(fa::DecodeParams);
+    if constexpr (FP8) kern = fa::fa_decode_fp8_kernel<RG, PAGED>;
+    else kern = fa::fa_decode_split_kernel<D, RG, PAGED>;
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
         bool &set = info->decode_attr_set[D == 128][RG == 8 ? 3 : RG == 4 ? 2 : RG == 2 ? 1 : 0][PAGED][FP8];
         if (!set) {
-            cudaError_t e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, RG, PAGED, FP8>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess)
                 return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
             set = true;
@@ -266,7 +274,7 @@ int launch_split(fa::DecodeParams p, DeviceInfo *info, cudaStream_t st)
     p.n_items = p.S_max * p.B * p.n_hg;
     const int max_ctas = fa::decode::kCtasPerSm * info->num_sms;
     const int grid = p.n_items < max_ctas ? p.n_items : max_ctas;
-    fa::fa_decode_split_kernel<D, RG, PAGED, FP8><<<grid, fa::decode::kThreads, C::kSmemBytes, st>>>(p);
+    kern<<<grid, fa::decode::kThreads, smem, st>>>(p);
     return FA_OK;
 }
 
@@ -361,8 +369,8 @@ int fa_decode(const void *q, const void *kcache, const void *vcache, const int *
     fa::DecodeParams p;
     memset(&p, 0, sizeof p);
     p.q = static_cast<const __nv_bfloat16 *>(q);
-    if ((rc = encode_rows_map(&p.tm_k, kcache, d, Nmax, (long long)B * Hkv, fa::decode::kSub)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_v, vcache, d, Nmax, (long long)B * Hkv, fa::decode::kSub)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_k, kcache, d, Nmax, (long long)B * Hkv, decode_block_keys(d, false))) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, vcache, d, Nmax, (long long)B * Hkv, decode_block_keys(d, false))) != FA_OK) return rc;
     p.seqlens = seqlens;
     p.S_max = (int)decode_splits(Nmax);
     p.part_o = static_cast<float *>(workspace);
@@ -450,15 +458,15 @@ int decode_general(const void *q, const CacheDesc &c, const int *seqlens, void *
     memset(&p, 0, sizeof p);
     p.q = static_cast<const __nv_bfloat16 *>(q);
     if (c.paged) {
-        // rows per copy: the largest power of two that divides page_size, at most 64
+        // rows per copy: the largest power of two that divides page_size, at most one block
         p.box_rows = c.page_size & -c.page_size;
-        if (p.box_rows > fa::decode::kSub) p.box_rows = fa::decode::kSub;
+        if (p.box_rows > decode_block_keys(d, c.fp8)) p.box_rows = decode_block_keys(d, c.fp8);
         p.block_table = c.block_table;
         p.page_size = c.page_size;
         p.max_pages = c.max_pages;
         p.num_pages = c.num_pages;
     } else {
-        p.box_rows = fa::decode::kSub;
+        p.box_rows = decode_block_keys(d, c.fp8);
     }
     const long long map_rows = c.paged ? c.page_size : Nmax;
     if ((rc = encode_rows_map(&p.tm_k, c.k, d, map_rows, planes, p.box_rows, c.fp8)) != FA_OK) return rc;
@@ -629,8 +637,8 @@ int fa_decode_noalloc(const void *q, const void *kcache, const void *vcache, con
     fa::DecodeParams p;
     memset(&p, 0, sizeof p);
     p.q = static_cast<const __nv_bfloat16 *>(q);
-    if ((rc = encode_rows_map(&p.tm_k, kcache, d, Nmax, (long long)B * Hkv, fa::decode::kSub)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_v, vcache, d, Nmax, (long long)B * Hkv, fa::decode::kSub)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_k, kcache, d, Nmax, (long long)B * Hkv, decode_block_keys(d, false))) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, vcache, d, Nmax, (long long)B * Hkv, decode_block_keys(d, false))) != FA_OK) return rc;
     p.seqlens = seqlens;
     p.S_max = (int)decode_splits(Nmax);
     p.part_o = static_cast<float *>(scratch);
