@@ -309,95 +309,6 @@ cudaError_t launch_merge(const fa::DecodeParams &p, cudaStream_t st)
 
 }  // namespace
 
-extern "C" {
-
-int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
-           int Hkv, int Nq, int Nk, int d, float scale, int causal, void *stream)
-{
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, stream, 0);
-}
-
-int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
-              int Hkv, int Nq, int Nk, int d, float scale, int causal, int o_dtype, void *stream)
-{
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, o_dtype, stream, 0);
-}
-
-int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse, int B,
-                  int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window, int o_dtype,
-                  void *stream)
-{
-    if (window <= 0) return fail(FA_ERR_INVALID, "window must be >= 1 (got %d)", window);
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, o_dtype, stream, 0);
-}
-
-int fa_fwd_selftest_timeout(const void *q, const void *k, const void *v, void *o, float *lse,
-                            int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
-                            int causal, void *stream)
-{
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, stream, 1);
-}
-
-size_t fa_decode_workspace_size(int B, int Hq, int Nmax, int d) { return decode_ws_bytes(B, Hq, Nmax, d); }
-
-int fa_decode(const void *q, const void *kcache, const void *vcache, const int *seqlens, void *o,
-              float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale, void *workspace,
-              size_t workspace_bytes, void *stream)
-{
-    if (!q || !kcache || !vcache || !seqlens || !o) return fail(FA_ERR_INVALID, "null pointer argument");
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nmax <= 0 || d <= 0)
-        return fail(FA_ERR_INVALID, "sizes must be positive (B=%d Hq=%d Hkv=%d Nmax=%d d=%d)", B, Hq, Hkv, Nmax, d);
-    if (Hq % Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
-    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(FA_ERR_INVALID, "scale must be finite and > 0");
-    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
-    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
-        return fail(FA_ERR_UNSUPPORTED, "q, kcache, vcache and o must be 16-byte aligned");
-    if (B > 65535 || decode_splits(Nmax) > 0x7fffffffLL)
-        return fail(FA_ERR_UNSUPPORTED, "B must be <= 65535");
-    const size_t need = decode_ws_bytes(B, Hq, Nmax, d);
-    if (!workspace || workspace_bytes < need)
-        return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
-    if (!aligned16(workspace)) return fail(FA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
-    int dev, rc;
-    DeviceInfo *info;
-    if ((rc = current_device(&dev, &info)) != FA_OK) return rc;
-
-    const int R = Hq / Hkv;
-    const int rg = (R % 8 == 0) ? 8 : (R % 4 == 0) ? 4 : (R % 2 == 0) ? 2 : 1;
-    if (Hq / rg > 65535) return fail(FA_ERR_UNSUPPORTED, "too many head groups");
-
-    fa::DecodeParams p;
-    memset(&p, 0, sizeof p);
-    p.q = static_cast<const __nv_bfloat16 *>(q);
-    if ((rc = encode_rows_map(&p.tm_k, kcache, d, Nmax, (long long)B * Hkv, decode_block_keys(d, false))) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_v, vcache, d, Nmax, (long long)B * Hkv, decode_block_keys(d, false))) != FA_OK) return rc;
-    p.seqlens = seqlens;
-    p.S_max = (int)decode_splits(Nmax);
-    p.part_o = static_cast<float *>(workspace);
-    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                           align256((size_t)B * Hq * p.S_max * d * sizeof(float)));
-    p.o = static_cast<__nv_bfloat16 *>(o);
-    p.lse = lse;
-    p.B = B;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.Nmax = Nmax;
-    p.R = R;
-    p.scale_log2 = scale * 1.4426950408889634f;
-
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    p.wait_limit_ns = g_wait_limit_ns;
-    rc = (d == 128) ? launch_split_rg<128>(p, rg, info, st) : launch_split_rg<64>(p, rg, info, st);
-    if (rc != FA_OK) return rc;
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
-    e = (d == 128) ? launch_merge<128>(p, st) : launch_merge<64>(p, st);
-    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
-    return ok();
-}
-
-}  // extern "C"
-
 namespace {
 
 // The caches of a decode call beyond the contiguous bf16 layout of fa_decode.
@@ -410,8 +321,8 @@ struct CacheDesc {
     int num_pages, page_size, max_pages;
 };
 
-// Validation and launch shared by the paged and the FP8 entry points.  Nmax is the
-// contiguous cache length (ignored when paged: page_size * max_pages).
+// Validation and launch shared by every decode entry point.  Nmax is the contiguous cache
+// length (ignored when paged: page_size * max_pages).
 int decode_general(const void *q, const CacheDesc &c, const int *seqlens, void *o, float *lse,
                    int B, int Hq, int Hkv, int Nmax, int d, float scale, void *workspace,
                    size_t workspace_bytes, void *stream, int o_dtype = FA_BF16)
@@ -507,6 +418,44 @@ int decode_general(const void *q, const CacheDesc &c, const int *seqlens, void *
 }  // namespace
 
 extern "C" {
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int d, float scale, int causal, void *stream)
+{
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, stream, 0);
+}
+
+int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+              int Hkv, int Nq, int Nk, int d, float scale, int causal, int o_dtype, void *stream)
+{
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, o_dtype, stream, 0);
+}
+
+int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                  int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window, int o_dtype,
+                  void *stream)
+{
+    if (window <= 0) return fail(FA_ERR_INVALID, "window must be >= 1 (got %d)", window);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, o_dtype, stream, 0);
+}
+
+int fa_fwd_selftest_timeout(const void *q, const void *k, const void *v, void *o, float *lse,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                            int causal, void *stream)
+{
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, stream, 1);
+}
+
+size_t fa_decode_workspace_size(int B, int Hq, int Nmax, int d) { return decode_ws_bytes(B, Hq, Nmax, d); }
+
+int fa_decode(const void *q, const void *kcache, const void *vcache, const int *seqlens, void *o,
+              float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale, void *workspace,
+              size_t workspace_bytes, void *stream)
+{
+    const CacheDesc c{kcache, vcache, false, nullptr, nullptr, false, nullptr, 0, 0, 0};
+    return decode_general(q, c, seqlens, o, lse, B, Hq, Hkv, Nmax, d, scale, workspace, workspace_bytes, stream);
+}
+
 
 int fa_decode_paged(const void *q, const void *kpages, const void *vpages, const int *block_table,
                     const int *seqlens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
@@ -608,60 +557,24 @@ int fa_decode_noalloc(const void *q, const void *kcache, const void *vcache, con
                       void *o, float *lse, int B, int Hq, int Hkv, int Nmax, int d, float scale,
                       void *stream)
 {
+    // the partials must fit the fixed scratch; every other check is fa_decode's
+    if (B > 0 && Hq > 0 && Nmax > 0 && d > 0) {
+        const size_t need = decode_ws_bytes(B, Hq, Nmax, d);
+        if (need > (size_t)FA_NOALLOC_SCRATCH_BYTES)
+            return fail(FA_ERR_WORKSPACE,
+                        "this decode needs %zu bytes of scratch; fa_decode_noalloc has %u bytes "
+                        "(use fa_decode with a workspace for larger problems)",
+                        need, (unsigned)FA_NOALLOC_SCRATCH_BYTES);
+    }
     if (!q || !kcache || !vcache || !seqlens || !o) return fail(FA_ERR_INVALID, "null pointer argument");
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nmax <= 0 || d <= 0)
-        return fail(FA_ERR_INVALID, "sizes must be positive (B=%d Hq=%d Hkv=%d Nmax=%d d=%d)", B, Hq, Hkv, Nmax, d);
-    if (Hq % Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
-    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(FA_ERR_INVALID, "scale must be finite and > 0");
-    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
-    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
-        return fail(FA_ERR_UNSUPPORTED, "q, kcache, vcache and o must be 16-byte aligned");
-    if (B > 65535 || decode_splits(Nmax) > 0x7fffffffLL)
-        return fail(FA_ERR_UNSUPPORTED, "B must be <= 65535");
-    const size_t need = decode_ws_bytes(B, Hq, Nmax, d);
-    if (need > (size_t)FA_NOALLOC_SCRATCH_BYTES)
-        return fail(FA_ERR_WORKSPACE,
-                    "this decode needs %zu bytes of scratch; fa_decode_noalloc has %u bytes "
-                    "(use fa_decode with a workspace for larger problems)",
-                    need, (unsigned)FA_NOALLOC_SCRATCH_BYTES);
     int dev, rc;
     DeviceInfo *info;
     if ((rc = current_device(&dev, &info)) != FA_OK) return rc;
     void *scratch = nullptr;
     if ((rc = noalloc_scratch(dev, &scratch)) != FA_OK) return rc;
-
-    const int R = Hq / Hkv;
-    const int rg = (R % 8 == 0) ? 8 : (R % 4 == 0) ? 4 : (R % 2 == 0) ? 2 : 1;
-    if (Hq / rg > 65535) return fail(FA_ERR_UNSUPPORTED, "too many head groups");
-
-    fa::DecodeParams p;
-    memset(&p, 0, sizeof p);
-    p.q = static_cast<const __nv_bfloat16 *>(q);
-    if ((rc = encode_rows_map(&p.tm_k, kcache, d, Nmax, (long long)B * Hkv, decode_block_keys(d, false))) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_v, vcache, d, Nmax, (long long)B * Hkv, decode_block_keys(d, false))) != FA_OK) return rc;
-    p.seqlens = seqlens;
-    p.S_max = (int)decode_splits(Nmax);
-    p.part_o = static_cast<float *>(scratch);
-    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(scratch) +
-                                           align256((size_t)B * Hq * p.S_max * d * sizeof(float)));
-    p.o = static_cast<__nv_bfloat16 *>(o);
-    p.lse = lse;
-    p.B = B;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.Nmax = Nmax;
-    p.R = R;
-    p.scale_log2 = scale * 1.4426950408889634f;
-
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    p.wait_limit_ns = g_wait_limit_ns;
-    rc = (d == 128) ? launch_split_rg<128>(p, rg, info, st) : launch_split_rg<64>(p, rg, info, st);
-    if (rc != FA_OK) return rc;
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode split launch: %s", cudaGetErrorString(e));
-    e = (d == 128) ? launch_merge<128>(p, st) : launch_merge<64>(p, st);
-    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
-    return ok();
+    const CacheDesc c{kcache, vcache, false, nullptr, nullptr, false, nullptr, 0, 0, 0};
+    return decode_general(q, c, seqlens, o, lse, B, Hq, Hkv, Nmax, d, scale, scratch,
+                          (size_t)FA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int fa_get_error(void *stream)

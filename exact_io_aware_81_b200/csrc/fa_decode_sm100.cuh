@@ -943,7 +943,8 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
 // One CTA of kMergeWarps warps per (query head, sequence).  Every warp finds the largest
 // partial log2-sum-exp M (lanes stride over the S partials); warp w then accumulates the
 // weighted partial outputs of splits w, w + kMergeWarps, ... with each lane owning D/32
-// consecutive elements; the warps' sums are added in shared memory.
+// consecutive elements (one vector load per split); the warps' sums are added in shared
+// memory.
 constexpr int kMergeWarps = 8;
 
 template <int D>
@@ -985,8 +986,17 @@ __global__ void __launch_bounds__(32 * kMergeWarps) fa_decode_merge_kernel(const
         const float w = ptx::ex2(pl[s] - M);
         den += w;
         const float *src = po + (size_t)s * D + lane * EPL;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+        if constexpr (EPL == 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(src);
+            acc[0] = fmaf(w, x.x, acc[0]);
+            acc[1] = fmaf(w, x.y, acc[1]);
+            acc[2] = fmaf(w, x.z, acc[2]);
+            acc[3] = fmaf(w, x.w, acc[3]);
+        } else {
+            const float2 x = *reinterpret_cast<const float2 *>(src);
+            acc[0] = fmaf(w, x.x, acc[0]);
+            acc[1] = fmaf(w, x.y, acc[1]);
+        }
     }
 #pragma unroll
     for (int e = 0; e < EPL; ++e) red[warp][lane * EPL + e] = acc[e];
