@@ -75,3 +75,18 @@ def test_lse_optional_and_workspace_reuse():
     torch.cuda.synchronize()
     assert l2 is None
     assert torch.equal(o1, o2)
+
+
+def test_many_sequences_with_empty_and_short_ones():
+    # more than 32 sequences: the work-item walk steps over the lengths 32 at a time
+    B = 100
+    w = inputs.make_decode(B, 8, 2, 700, 128, seed=12, len_range=(0, 700))
+    g = torch.Generator().manual_seed(13)
+    sl = torch.randint(0, 701, (B,), generator=g).to(torch.int32)
+    sl[::7] = 0
+    sl[3::11] = 1
+    sl[5::13] = 700
+    o, lse, status = run_gpu(w, sl)
+    assert status == ops.FA_OK
+    ro, rl = oracle.decode(w.q, w.kcache, w.vcache, sl, w.scale)
+    compare(o, lse, ro, rl, "many sequences")

@@ -115,3 +115,16 @@ def test_paged_fp8_equals_contiguous(ps):
     assert torch.equal(o, oc) and torch.equal(lse, lc)
     ro, rl = oracle.decode_fp8(w.q, w.kcache, w.vcache, w.k_scale, w.v_scale, sl, w.scale)
     compare(o, lse, ro, rl, f"paged fp8 {ps}")
+
+
+def test_fp8_many_sequences():
+    # more than 32 sequences and more items than the kernel has workers
+    B = 100
+    w = inputs.make_fp8_decode(B, 8, 2, 1000, 128, seed=35, len_range=(0, 1000))
+    sl = w.seqlens.clone()
+    sl[::9] = 0
+    sl[2::10] = 1
+    o, lse, status = run_fp8(w, sl)
+    assert status == ops.FA_OK
+    ro, rl = oracle.decode_fp8(w.q, w.kcache, w.vcache, w.k_scale, w.v_scale, sl, w.scale)
+    compare(o, lse, ro, rl, "fp8 many sequences")

@@ -110,3 +110,12 @@ def test_paged_seqlen_out_of_range_is_clamped_and_reported():
     ro, rl = oracle.decode_paged(w.q, w.kpages, w.vpages, w.block_table,
                                  torch.tensor([64, 0], dtype=torch.int32), w.scale)
     compare(o, lse, ro, rl, "clamped")
+
+
+def test_paged_many_sequences():
+    # more than 32 sequences, some empty, pages scattered over the pool
+    w = inputs.make_paged_decode(90, 8, 2, 32, 20, 128, seed=15, len_range=(0, 640))
+    o, lse, status = run_paged(w.q, w.kpages, w.vpages, w.block_table, w.seqlens, w.scale)
+    assert status == ops.FA_OK
+    ro, rl = oracle.decode_paged(w.q, w.kpages, w.vpages, w.block_table, w.seqlens, w.scale)
+    compare(o, lse, ro, rl, "paged many sequences")
