@@ -29,28 +29,10 @@ struct StopFlag {
     __device__ __forceinline__ void stop() const { *flag = 1; }
 };
 
-// Wait by one thread for the phase of `bar` with parity `parity`.  Returns false if the
-// CTA was told to stop or the limit ran out (which records kErrTimeout and tells the
-// CTA to stop).
-__device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t parity, const StopFlag &sf)
-{
-    if (ptx::mbar_test(bar, parity)) return true;
-    const uint64_t t0 = ptx::globaltimer_ns();
-    for (uint32_t n = 1;; ++n) {
-        if (ptx::mbar_test(bar, parity)) return true;
-        if ((n & 31u) == 0u) {
-            if (sf.stopped()) return false;
-            if (ptx::globaltimer_ns() - t0 > sf.limit_ns) {
-                raise_error(kErrTimeout);
-                sf.stop();
-                return false;
-            }
-        }
-    }
-}
-
-// The same wait made by all 32 lanes of a warp together; the outcome is warp-uniform,
-// so that warp-collective tensor-memory instructions after it stay converged.
+// Wait, by all 32 lanes of a warp together, for the phase of `bar` with parity `parity`.
+// Returns false if the CTA was told to stop or the limit ran out (which records
+// kErrTimeout and tells the CTA to stop).  The outcome is warp-uniform, so that
+// warp-collective tensor-memory instructions after it stay converged.
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const StopFlag &sf)
 {
     if (__all_sync(0xffffffffu, ptx::mbar_test(bar, parity))) return true;

@@ -95,17 +95,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
-// 1-D bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global
-// to shared memory; completion is counted in bytes on `bar`.
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_addr(dst)),
-        "l"(src), "r"(bytes), "r"(smem_addr(bar))
-        : "memory");
-}
-
 // 3-D tiled store of one box from shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int x, int y, int z)
 {
@@ -122,12 +111,6 @@ __device__ __forceinline__ void bulk_wait_group_read0() { asm volatile("cp.async
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Order this thread's generic-proxy shared-memory writes before later async-proxy reads.
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-// Barrier among COUNT threads (a multiple of 32) on hardware barrier ID (1..15).
-template <int ID, int COUNT>
-__device__ __forceinline__ void named_barrier_sync()
-{
-    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(COUNT) : "memory");
-}
 
 // -------------------------------------------------------------------- tensor memory
 
