@@ -427,30 +427,36 @@ def run_ours(args, rank, world, local):
 
 def run_extra(args, dev, peaks):
     """Per-workload kernel times for the other workloads (not part of the step): the other
-    causal shapes, sliding window (6, 8), chunked prefill (7, 8), paged decode (9) and FP8
-    decode (10).  Caches of decode 9 and 10 (over 1 GB) exceed L2; prefill 1 does not."""
+    causal shapes, prefill 3 on (batch, sequence, heads, dim) tensors (fa_fwd_bshd), sliding
+    window (6, 8), chunked prefill (7, 8), paged decode (9) and FP8 decode (10).  Caches of
+    decode 9 and 10 (over 1 GB) exceed L2; prefill 1 does not."""
     from exact_io_aware_81_b200 import ops
     res = {}
-    for kid in (1, 3, 4, 6, 7, 8):
+    for kid, bshd in ((1, False), (3, False), (3, True), (4, False), (6, False), (7, False), (8, False)):
         w = inputs.workload(kid)
         B, Hq, Hkv, Nq, Nk, d = w.shape
-        q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
-        o = torch.empty((B, Hq, Nq, d), dtype=w.out_dtype, device=dev)
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+        if bshd:
+            q, k, v = (t.transpose(1, 2).contiguous().to(dev) for t in (w.q, w.k, w.v))
+            o = torch.empty((B, Nq, Hq, d), dtype=w.out_dtype, device=dev)
+            fwd = ops.fwd_bshd
+        else:
+            q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+            o = torch.empty((B, Hq, Nq, d), dtype=w.out_dtype, device=dev)
+            fwd = ops.fwd
         n = 3 if kid != 1 else 20
         for _ in range(3):
-            ops.fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse,
-                    window=w.window)
+            fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse, window=w.window)
         e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         e[0].record()
         for _ in range(n):
-            ops.fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse,
-                    window=w.window)
+            fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse, window=w.window)
         e[1].record()
         torch.cuda.synchronize(dev)
         ms = e[0].elapsed_time(e[1]) / n
         tf = w.flops() / (ms * 1e-3) / 1e12
-        res[w.name] = {"ms": ms, "tflops": tf, "frac": tf / peaks.get("bf16_tflops", 1590.0)}
+        res[w.name + ("_bshd" if bshd else "")] = {"ms": ms, "tflops": tf,
+                                                   "frac": tf / peaks.get("bf16_tflops", 1590.0)}
         del q, k, v, o, lse
         torch.cuda.empty_cache()
     # decode over a paged cache (9) and over an FP8 cache (10): HBM-bound like decode 5

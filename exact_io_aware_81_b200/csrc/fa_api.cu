@@ -120,6 +120,26 @@ int encode_rows_map(CUtensorMap *m, const void *base, int D, long long rows, lon
     return FA_OK;
 }
 
+// A prefill operand as a 4-D (d, rows, heads, batch) bf16 tensor with boxes of `box_rows`
+// rows x 64 columns of one head, 128-byte swizzle.  The memory layout is (batch, heads,
+// rows, d), or (batch, rows, heads, d) when `bshd`: only the strides differ.
+int encode_heads_map(CUtensorMap *m, const void *base, int D, int rows, int heads, int batch, bool bshd,
+                     unsigned box_rows = 128)
+{
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t row = (cuuint64_t)D * 2, plane = (cuuint64_t)rows * heads * row;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)batch};
+    cuuint64_t strides[3] = {bshd ? heads * row : row, bshd ? row : rows * row, plane};
+    cuuint32_t box[4] = {64, box_rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return FA_OK;
+}
+
 // ------------------------------------------------------------------- prefill
 
 int validate_fwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
@@ -178,7 +198,7 @@ int launch_prefill_variant(const fa::PrefillParams &p, DeviceInfo *info, cudaStr
 
 int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
              int Hkv, int Nq, int Nk, int d, float scale, int causal, int window, int o_dtype,
-             void *stream, int selftest_timeout)
+             bool bshd, void *stream, int selftest_timeout)
 {
     int rc = validate_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, o_dtype);
     if (rc != FA_OK) return rc;
@@ -190,11 +210,14 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
 
     fa::PrefillParams p;
     memset(&p, 0, sizeof p);
-    if ((rc = encode_rows_map(&p.tm_q, q, d, Nq, (long long)B * Hq)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_k, k, d, Nk, (long long)B * Hkv)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_v, v, d, Nk, (long long)B * Hkv)) != FA_OK) return rc;
-    if (o_dtype == FA_BF16 && (rc = encode_rows_map(&p.tm_o, o, d, Nq, (long long)B * Hq, 32)) != FA_OK) return rc;
+    if ((rc = encode_heads_map(&p.tm_q, q, d, Nq, Hq, B, bshd)) != FA_OK) return rc;
+    if ((rc = encode_heads_map(&p.tm_k, k, d, Nk, Hkv, B, bshd)) != FA_OK) return rc;
+    if ((rc = encode_heads_map(&p.tm_v, v, d, Nk, Hkv, B, bshd)) != FA_OK) return rc;
+    if (o_dtype == FA_BF16 && (rc = encode_heads_map(&p.tm_o, o, d, Nq, Hq, B, bshd, 32)) != FA_OK) return rc;
     p.o = o;
+    p.o_sb = (long long)Hq * Nq * d;
+    p.o_sh = bshd ? d : (long long)Nq * d;
+    p.o_sn = bshd ? (long long)Hq * d : d;
     p.lse = lse;
     p.B = B;
     p.Hq = Hq;
@@ -422,13 +445,13 @@ extern "C" {
 int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
            int Hkv, int Nq, int Nk, int d, float scale, int causal, void *stream)
 {
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, stream, 0);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, false, stream, 0);
 }
 
 int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
               int Hkv, int Nq, int Nk, int d, float scale, int causal, int o_dtype, void *stream)
 {
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, o_dtype, stream, 0);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, o_dtype, false, stream, 0);
 }
 
 int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse, int B,
@@ -436,14 +459,21 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *l
                   void *stream)
 {
     if (window <= 0) return fail(FA_ERR_INVALID, "window must be >= 1 (got %d)", window);
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, o_dtype, stream, 0);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, o_dtype, false, stream, 0);
+}
+
+int fa_fwd_bshd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int d, float scale, int causal, int window, int o_dtype,
+                void *stream)
+{
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, o_dtype, true, stream, 0);
 }
 
 int fa_fwd_selftest_timeout(const void *q, const void *k, const void *v, void *o, float *lse,
                             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
                             int causal, void *stream)
 {
-    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, stream, 1);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, false, stream, 1);
 }
 
 size_t fa_decode_workspace_size(int B, int Hq, int Nmax, int d) { return decode_ws_bytes(B, Hq, Nmax, d); }

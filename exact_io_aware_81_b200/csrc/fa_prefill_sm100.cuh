@@ -44,11 +44,14 @@
 namespace fa {
 
 struct PrefillParams {
-    CUtensorMap tm_q;  // (d, Nq, B*Hq) bf16, box (64, 128, 1), 128B swizzle
-    CUtensorMap tm_k;  // (d, Nk, B*Hkv)
-    CUtensorMap tm_v;  // (d, Nk, B*Hkv)
-    CUtensorMap tm_o;  // (d, Nq, B*Hq) bf16 output, box (64, 32, 1), 128B swizzle: one warp's rows
+    // The maps view every tensor as 4-D (d, rows, heads, batch) whatever its layout in memory
+    // ((B, H, N, d) or (B, N, H, d)): only the strides differ.
+    CUtensorMap tm_q;  // (d, Nq, Hq, B) bf16, box (64, 128, 1, 1), 128B swizzle
+    CUtensorMap tm_k;  // (d, Nk, Hkv, B)
+    CUtensorMap tm_v;  // (d, Nk, Hkv, B)
+    CUtensorMap tm_o;  // (d, Nq, Hq, B) bf16 output, box (64, 32, 1, 1), 128B swizzle: one warp's rows
     void *o;
+    long long o_sb, o_sh, o_sn;  // fp32 output: element strides of batch, head and row
     float *lse;
     int B, Hq, Hkv, Nq, Nk;
     int R;           // Hq / Hkv
@@ -394,8 +397,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 uint8_t *dst = smem + C::kQOff + qi * C::kTileBytes;
 #pragma unroll
                 for (int c = 0; c < D / 64; ++c)
-                    ptx::tma_load_3d(dst + c * kChunkBytes, &p.tm_q, &q_full[qi], 64 * c, r,
-                                     uw.b * p.Hq + h);
+                    ptx::tma_load_4d(dst + c * kChunkBytes, &p.tm_q, &q_full[qi], 64 * c, r, h, uw.b);
             }
             __syncwarp();
         };
@@ -411,7 +413,6 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         for (; ok && u >= 0; ++i) {
             const int un = next_unit<WINDOW>(p, unit_step(u), wn);
             int q_next = (un >= 0) ? 0 : 2;  // look-ahead Q tiles already issued
-            const int plane = w.b * p.Hkv + w.g;
             for (int j = w.a0; j < w.n1 && ok; ++j) {
                 for (int kv = 0; kv < 2; ++kv) {
                     const uint32_t st = kv_it % C::kStages;
@@ -423,8 +424,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                         const CUtensorMap *map = kv ? &p.tm_v : &p.tm_k;
 #pragma unroll
                         for (int c = 0; c < D / 64; ++c)
-                            ptx::tma_load_3d(dst + c * kChunkBytes, map, &kv_full[st], 64 * c,
-                                             BN * j, plane);
+                            ptx::tma_load_4d(dst + c * kChunkBytes, map, &kv_full[st], 64 * c, BN * j, w.g, w.b);
                     }
                     __syncwarp();
                     ++kv_it;
@@ -683,7 +683,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             ptx::tc_fence_after();
             const bool valid = row < p.Nq;
             const float inv_l = 1.f / lo;
-            const size_t orow = ((size_t)w.b * p.Hq + h) * (size_t)p.Nq + (size_t)(valid ? row : 0);
+            const size_t orow = ((size_t)w.b * p.Hq + h) * (size_t)p.Nq + (size_t)(valid ? row : 0);  // LSE index
             const int qi = 2 * (int)(units & 1u) + s;
             uint32_t ov[D];
 #pragma unroll
@@ -693,7 +693,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             ptx::mbar_arrive(&o_free[s]);
             if (OUT_F32) {
                 if (valid) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D);
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + w.b * p.o_sb + h * p.o_sh +
+                                                             (long long)row * p.o_sn);
 #pragma unroll
                     for (int e = 0; e < D / 4; ++e)
                         dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
@@ -722,8 +723,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     if (r0 + wr < p.Nq) {            // (rows past Nq are never stored)
 #pragma unroll
                         for (int c = 0; c < D / 64; ++c)
-                            ptx::tma_store_3d(&p.tm_o, stage + c * kChunkBytes + wr * 128, 64 * c, r0 + wr,
-                                              w.b * p.Hq + h);
+                            ptx::tma_store_4d(&p.tm_o, stage + c * kChunkBytes + wr * 128, 64 * c, r0 + wr, h, w.b);
                         ptx::bulk_commit_group();
                         ptx::bulk_wait_group_read0();
                     }

@@ -34,6 +34,7 @@ SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "fa_fwd_bshd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
     "fa_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
@@ -107,6 +108,17 @@ def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _output(t: Optional[torch.Tensor], name: str, dtype: torch.dtype, shape, device) -> torch.Tensor:
+    """A caller-provided output checked against its dtype and exact shape, or a new one."""
+    shape = tuple(shape)
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    _require(t, name, dtype, len(shape))
+    if tuple(t.shape) != shape:
+        raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+    return t
+
+
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale: Optional[float] = None, out_dtype: torch.dtype = torch.bfloat16,
         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
@@ -130,14 +142,7 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale = 1.0 / math.sqrt(d)
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out_dtype must be bfloat16 or float32")
-    if out is None:
-        out = torch.empty((B, Hq, Nq, d), dtype=out_dtype, device=q.device)
-    else:
-        _require(out, "out", out_dtype, 4)
-    if lse is None:
-        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-    else:
-        _require(lse, "lse", torch.float32, 3)
+    out, lse = _fwd_outputs(q, (B, Hq, Nq, d), (B, Hq, Nq), out_dtype, out, lse)
     odt = FA_F32 if out_dtype == torch.float32 else FA_BF16
     if window:
         if not causal:
@@ -149,6 +154,40 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         rc = load().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                               lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
                               odt, _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def _fwd_outputs(q, o_shape, lse_shape, out_dtype, out, lse):
+    return (_output(out, "out", out_dtype, o_shape, q.device),
+            _output(lse, "lse", torch.float32, lse_shape, q.device))
+
+
+def fwd_bshd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+             scale: Optional[float] = None, out_dtype: torch.dtype = torch.bfloat16,
+             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+             stream=None, window: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Attention forward on (batch, sequence, heads, dim) tensors (fa_fwd_bshd), the layout
+    flash_attn_func takes: q (B,Nq,Hq,d), k/v (B,Nk,Hkv,d) bf16 -> o (B,Nq,Hq,d) and lse
+    fp32 (B,Hq,Nq).  causal, scale, window and out_dtype as fwd."""
+    _require(q, "q", torch.bfloat16, 4)
+    _require(k, "k", torch.bfloat16, 4)
+    _require(v, "v", torch.bfloat16, 4)
+    B, Nq, Hq, d = q.shape
+    Bk, Nk, Hkv, dk = k.shape
+    if (Bk, dk) != (B, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k.shape)} v {tuple(v.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    if window and not causal:
+        raise ValueError("a sliding window needs causal=True")
+    out, lse = _fwd_outputs(q, (B, Nq, Hq, d), (B, Hq, Nq), out_dtype, out, lse)
+    odt = FA_F32 if out_dtype == torch.float32 else FA_BF16
+    rc = load().fa_fwd_bshd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                            B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), int(window), odt,
+                            _stream_handle(stream))
     _check(rc)
     return out, lse
 
@@ -193,14 +232,7 @@ def decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     elif not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
-    else:
-        _require(out, "out", torch.bfloat16, 3)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    elif lse is not None:
-        _require(lse, "lse", torch.float32, 2)
+    out, lse = _decode_outputs(q, out, lse, want_lse)
     rc = load().fa_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
                           out.data_ptr(), lse.data_ptr() if lse is not None else None,
                           B, Hq, Hkv, Nmax, d, float(scale), workspace.data_ptr(),
@@ -235,14 +267,7 @@ def decode_paged(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor,
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     elif not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
-    else:
-        _require(out, "out", torch.bfloat16, 3)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    elif lse is not None:
-        _require(lse, "lse", torch.float32, 2)
+    out, lse = _decode_outputs(q, out, lse, want_lse)
     rc = load().fa_decode_paged(q.data_ptr(), kpages.data_ptr(), vpages.data_ptr(),
                                 block_table.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
                                 lse.data_ptr() if lse is not None else None, B, Hq, Hkv,
@@ -253,16 +278,11 @@ def decode_paged(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor,
     return out, lse
 
 
-def _decode_outputs(q, out, lse, want_lse):
+def _decode_outputs(q, out, lse, want_lse, out_dtype=torch.bfloat16):
     B, Hq, d = q.shape
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
-    else:
-        _require(out, "out", torch.bfloat16, 3)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    elif lse is not None:
-        _require(lse, "lse", torch.float32, 2)
+    out = _output(out, "out", out_dtype, (B, Hq, d), q.device)
+    if lse is not None or want_lse:
+        lse = _output(lse, "lse", torch.float32, (B, Hq), q.device)
     return out, lse
 
 
@@ -293,14 +313,7 @@ def decode_ex(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqle
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     workspace = _workspace(workspace, decode_workspace_size(B, Hq, Nmax, d), q.device)
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=out_dtype, device=q.device)
-    else:
-        _require(out, "out", out_dtype, 3)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    elif lse is not None:
-        _require(lse, "lse", torch.float32, 2)
+    out, lse = _decode_outputs(q, out, lse, want_lse, out_dtype)
     rc = load().fa_decode_ex(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
                              out.data_ptr(), lse.data_ptr() if lse is not None else None,
                              B, Hq, Hkv, Nmax, d, float(scale),
@@ -325,12 +338,8 @@ def merge_lse(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype: torch.d
         rows *= x
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out_dtype must be bfloat16 or float32")
-    if out is None:
-        out = torch.empty(row_shape + (d,), dtype=out_dtype, device=o_parts.device)
-    else:
-        _require(out, "out", out_dtype, len(row_shape) + 1)
-    if lse is None:
-        lse = torch.empty(row_shape, dtype=torch.float32, device=o_parts.device)
+    out = _output(out, "out", out_dtype, row_shape + (d,), o_parts.device)
+    lse = _output(lse, "lse", torch.float32, row_shape, o_parts.device)
     rc = load().fa_merge_lse(o_parts.data_ptr(), lse_parts.data_ptr(), P, rows, d, out.data_ptr(),
                              lse.data_ptr(), FA_F32 if out_dtype == torch.float32 else FA_BF16,
                              _stream_handle(stream))
@@ -450,9 +459,7 @@ def decode_noalloc(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor,
         scale = 1.0 / math.sqrt(d)
     if out is None:
         raise ValueError("decode_noalloc writes into a caller-provided `out`")
-    _require(out, "out", torch.bfloat16, 3)
-    if lse is not None:
-        _require(lse, "lse", torch.float32, 2)
+    out, lse = _decode_outputs(q, out, lse, False)
     rc = load().fa_decode_noalloc(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
                                   seqlens.data_ptr(), out.data_ptr(),
                                   lse.data_ptr() if lse is not None else None,

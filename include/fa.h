@@ -90,6 +90,24 @@ FA_API int fa_fwd_window(const void *q, const void *k, const void *v, void *o, f
                   int o_dtype, void *stream);
 
 /*
+ * Forward attention on (batch, sequence, heads, dim) tensors, the layout of the
+ * flash_attn_func call in toolsku.com "attention mechanism evolution", FlashAttention
+ * usage example (its layer views the projections as (B, S, H, d) and passes them on with
+ * no transpose):
+ *   q   (B, Nq, Hq,  d) bf16          k, v (B, Nk, Hkv, d) bf16
+ *   o   (B, Nq, Hq,  d) written, bf16 or fp32 (o_dtype)
+ *   lse (B, Hq,  Nq)    fp32 written (the head-major layout of fa_fwd)
+ *   causal, scale: as fa_fwd.  window: 0 for none, else W >= 1 with causal != 0, as
+ *   fa_fwd_window (FA_ERR_INVALID for W < 0 or a window without causal).
+ * The result equals fa_fwd_ex / fa_fwd_window on the same tensors transposed to
+ * (B, H, N, d): the kernel reads the same tiles through strided TMA descriptors, so no
+ * transposed copy is made.  Supported sizes and errors as fa_fwd_ex.
+ */
+FA_API int fa_fwd_bshd(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                int window, int o_dtype, void *stream);
+
+/*
  * Bytes of device workspace fa_decode needs for these sizes (fp32 partial outputs and
  * partial log-sum-exps of the split-KV chunks).  0 if the sizes are invalid.
  */

@@ -230,3 +230,25 @@ def test_decode_ex_rejects(lib):
     assert rc == ops.FA_ERR_INVALID                  # unknown output dtype
     rc = lib.fa_decode_ex(FAKE, FAKE, FAKE, None, FAKE, None, 2, 8, 2, 300, 128, 0.1, 1, FAKE, ws, None)
     assert rc == ops.FA_ERR_INVALID                  # no seqlens
+
+
+def _fwd_bshd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=4, Hkv=2, Nq=8, Nk=8, d=64,
+             scale=0.125, causal=1, window=0, dt=0)
+    a.update(kw)
+    return lib.fa_fwd_bshd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                           a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"], a["window"], a["dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(window=-1), ops.FA_ERR_INVALID),
+    (dict(causal=0, window=4), ops.FA_ERR_INVALID),    # a window needs causal attention
+    (dict(Nq=9, Nk=8), ops.FA_ERR_INVALID),
+    (dict(Hq=6, Hkv=4), ops.FA_ERR_INVALID),
+    (dict(dt=3), ops.FA_ERR_INVALID),
+    (dict(d=96), ops.FA_ERR_UNSUPPORTED),
+    (dict(k=FAKE + 8), ops.FA_ERR_UNSUPPORTED),
+])
+def test_fwd_bshd_rejects(lib, kw, status):
+    assert _fwd_bshd(lib, **kw) == status
+
