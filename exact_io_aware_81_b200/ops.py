@@ -8,6 +8,7 @@ raises instead of falling back to anything else.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -89,10 +90,22 @@ def _check(rc: int):
         raise FAError(rc, load().fa_last_error_message().decode())
 
 
-def _stream_handle(stream) -> int:
+def _stream_handle(stream, device=None) -> int:
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return int(stream.cuda_stream)
+
+
+@contextlib.contextmanager
+def _on_device(*tensors):
+    """Run a library call on the device of its tensors (the C ABI launches on the current
+    device); every tensor passed must be on that one device."""
+    dev = tensors[0].device
+    for t in tensors[1:]:
+        if t is not None and t.device != dev:
+            raise ValueError(f"all tensors must be on {dev}; found one on {t.device}")
+    with torch.cuda.device(dev):
+        yield dev
 
 
 def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
@@ -147,13 +160,15 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     if window:
         if not causal:
             raise ValueError("a sliding window needs causal=True")
-        rc = load().fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                  lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(window),
-                                  odt, _stream_handle(stream))
+        with _on_device(q, k, v, out, lse) as dev:
+            rc = load().fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                      lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(window),
+                                      odt, _stream_handle(stream, dev))
     else:
-        rc = load().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                              lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
-                              odt, _stream_handle(stream))
+        with _on_device(q, k, v, out, lse) as dev:
+            rc = load().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+                                  odt, _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 
@@ -185,9 +200,10 @@ def fwd_bshd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
         raise ValueError("a sliding window needs causal=True")
     out, lse = _fwd_outputs(q, (B, Nq, Hq, d), (B, Hq, Nq), out_dtype, out, lse)
     odt = FA_F32 if out_dtype == torch.float32 else FA_BF16
-    rc = load().fa_fwd_bshd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                            B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), int(window), odt,
-                            _stream_handle(stream))
+    with _on_device(q, k, v, out, lse) as dev:
+        rc = load().fa_fwd_bshd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), int(window), odt,
+                                _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 
@@ -233,10 +249,11 @@ def decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens:
     elif not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     out, lse = _decode_outputs(q, out, lse, want_lse)
-    rc = load().fa_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
-                          out.data_ptr(), lse.data_ptr() if lse is not None else None,
-                          B, Hq, Hkv, Nmax, d, float(scale), workspace.data_ptr(),
-                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    with _on_device(q, kcache, vcache, seqlens, out, lse, workspace) as dev:
+        rc = load().fa_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
+                              out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                              B, Hq, Hkv, Nmax, d, float(scale), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 
@@ -268,12 +285,13 @@ def decode_paged(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor,
     elif not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     out, lse = _decode_outputs(q, out, lse, want_lse)
-    rc = load().fa_decode_paged(q.data_ptr(), kpages.data_ptr(), vpages.data_ptr(),
-                                block_table.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
-                                lse.data_ptr() if lse is not None else None, B, Hq, Hkv,
-                                num_pages, page_size, max_pages, d, float(scale),
-                                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                _stream_handle(stream))
+    with _on_device(q, kpages, vpages, block_table, seqlens, out, lse, workspace) as dev:
+        rc = load().fa_decode_paged(q.data_ptr(), kpages.data_ptr(), vpages.data_ptr(),
+                                    block_table.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr() if lse is not None else None, B, Hq, Hkv,
+                                    num_pages, page_size, max_pages, d, float(scale),
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 
@@ -314,11 +332,12 @@ def decode_ex(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqle
         scale = 1.0 / math.sqrt(d)
     workspace = _workspace(workspace, decode_workspace_size(B, Hq, Nmax, d), q.device)
     out, lse = _decode_outputs(q, out, lse, want_lse, out_dtype)
-    rc = load().fa_decode_ex(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
-                             out.data_ptr(), lse.data_ptr() if lse is not None else None,
-                             B, Hq, Hkv, Nmax, d, float(scale),
-                             FA_F32 if out_dtype == torch.float32 else FA_BF16, workspace.data_ptr(),
-                             workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    with _on_device(q, kcache, vcache, seqlens, out, lse, workspace) as dev:
+        rc = load().fa_decode_ex(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
+                                 out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                 B, Hq, Hkv, Nmax, d, float(scale),
+                                 FA_F32 if out_dtype == torch.float32 else FA_BF16, workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 
@@ -340,9 +359,10 @@ def merge_lse(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype: torch.d
         raise ValueError("out_dtype must be bfloat16 or float32")
     out = _output(out, "out", out_dtype, row_shape + (d,), o_parts.device)
     lse = _output(lse, "lse", torch.float32, row_shape, o_parts.device)
-    rc = load().fa_merge_lse(o_parts.data_ptr(), lse_parts.data_ptr(), P, rows, d, out.data_ptr(),
-                             lse.data_ptr(), FA_F32 if out_dtype == torch.float32 else FA_BF16,
-                             _stream_handle(stream))
+    with _on_device(o_parts, lse_parts, out, lse) as dev:
+        rc = load().fa_merge_lse(o_parts.data_ptr(), lse_parts.data_ptr(), P, rows, d, out.data_ptr(),
+                                 lse.data_ptr(), FA_F32 if out_dtype == torch.float32 else FA_BF16,
+                                 _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 
@@ -368,11 +388,12 @@ def decode_fp8(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, k_sc
         scale = 1.0 / math.sqrt(d)
     workspace = _workspace(workspace, decode_workspace_size(B, Hq, Nmax, d), q.device)
     out, lse = _decode_outputs(q, out, lse, want_lse)
-    rc = load().fa_decode_fp8(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), k_scale.data_ptr(),
-                              v_scale.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
-                              lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nmax, d,
-                              float(scale), workspace.data_ptr(),
-                              workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    with _on_device(q, kcache, vcache, k_scale, v_scale, seqlens, out, lse, workspace) as dev:
+        rc = load().fa_decode_fp8(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), k_scale.data_ptr(),
+                                  v_scale.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
+                                  lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nmax, d,
+                                  float(scale), workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(), _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 
@@ -401,13 +422,14 @@ def decode_paged_fp8(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor
         scale = 1.0 / math.sqrt(d)
     workspace = _workspace(workspace, decode_workspace_size(B, Hq, page_size * max_pages, d), q.device)
     out, lse = _decode_outputs(q, out, lse, want_lse)
-    rc = load().fa_decode_paged_fp8(q.data_ptr(), kpages.data_ptr(), vpages.data_ptr(),
-                                    k_scale.data_ptr(), v_scale.data_ptr(), block_table.data_ptr(),
-                                    seqlens.data_ptr(), out.data_ptr(),
-                                    lse.data_ptr() if lse is not None else None, B, Hq, Hkv,
-                                    num_pages, page_size, max_pages, d, float(scale),
-                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                    _stream_handle(stream))
+    with _on_device(q, kpages, vpages, k_scale, v_scale, block_table, seqlens, out, lse, workspace) as dev:
+        rc = load().fa_decode_paged_fp8(q.data_ptr(), kpages.data_ptr(), vpages.data_ptr(),
+                                        k_scale.data_ptr(), v_scale.data_ptr(), block_table.data_ptr(),
+                                        seqlens.data_ptr(), out.data_ptr(),
+                                        lse.data_ptr() if lse is not None else None, B, Hq, Hkv,
+                                        num_pages, page_size, max_pages, d, float(scale),
+                                        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                        _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 
@@ -429,9 +451,10 @@ def fwd_selftest_timeout(q, k, v, causal=False, scale=None, stream=None):
         scale = 1.0 / math.sqrt(d)
     out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-    rc = load().fa_fwd_selftest_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                        lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
-                                        int(bool(causal)), _stream_handle(stream))
+    with _on_device(q, k, v, out, lse) as dev:
+        rc = load().fa_fwd_selftest_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                            lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                            int(bool(causal)), _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 
@@ -460,9 +483,10 @@ def decode_noalloc(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor,
     if out is None:
         raise ValueError("decode_noalloc writes into a caller-provided `out`")
     out, lse = _decode_outputs(q, out, lse, False)
-    rc = load().fa_decode_noalloc(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
-                                  seqlens.data_ptr(), out.data_ptr(),
-                                  lse.data_ptr() if lse is not None else None,
-                                  B, Hq, Hkv, Nmax, d, float(scale), _stream_handle(stream))
+    with _on_device(q, kcache, vcache, seqlens, out, lse) as dev:
+        rc = load().fa_decode_noalloc(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
+                                      seqlens.data_ptr(), out.data_ptr(),
+                                      lse.data_ptr() if lse is not None else None,
+                                      B, Hq, Hkv, Nmax, d, float(scale), _stream_handle(stream, dev))
     _check(rc)
     return out, lse
