@@ -8,6 +8,16 @@ GB/s is in ``decode``.  Timing: CUDA events on the launching stream, W untimed w
 steps, K timed steps bracketed by a barrier and a synchronize, max over ranks.  Both
 workloads' inputs exceed the 126 MB L2, so no flush is needed between steps.
 
+The same line carries a ``configs`` block: every other named workload (the grouped-query
+causal prefills at 8K and 32K, the same 8K problem on (batch, sequence, heads, dim) tensors,
+sliding window, chunked prefill, paged and FP8 decode, and the small fp32-output problem)
+timed the same way, one kernel call per timed iteration, with its roofline fraction.
+
+``--gpus N``: one process per GPU.  Under torchrun the world size must equal N; started
+without torchrun, the script re-launches itself under ``torch.distributed.run`` with N local
+ranks.  Every rank runs the same step on its own replica of the workload (no collective on
+the data path); times are the max over ranks.
+
 ``--impl reference`` times the CPU fp64 oracle (the only reference this method has) on a
 bounded row sample of the same prefill workload, on the host cores, with the same metric.
 """
@@ -151,12 +161,31 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ helpers
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def relaunch_cmd(n: int, argv, port: int):
+    """The torchrun command that starts this script as n local ranks with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}: start one process per GPU "
+                         f"(torchrun --nproc-per-node {args.gpus}), or run without torchrun and let "
+                         f"--gpus start the ranks")
     if args.impl == "reference":
         return rank, world, local  # the CPU oracle needs no process group
+    if local >= torch.cuda.device_count():
+        raise SystemExit(f"bench.py: local rank {local} has no GPU ({torch.cuda.device_count()} visible)")
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -418,20 +447,41 @@ def run_ours(args, rank, world, local):
         "gpu_launches": 3 * args.steps,
         "gpu": torch.cuda.get_device_name(dev),
     }
-    if args.extra:
-        result["extra"] = run_extra(args, dev, peaks)
+    if not args.no_configs:
+        result["configs"] = run_configs(dev, peaks, world)
+        result["gpu_launches"] += result["configs"].pop("_launches")
     if rank == 0:
         print(json.dumps(result), flush=True)
     return result
 
 
-def run_extra(args, dev, peaks):
-    """Per-workload kernel times for the other workloads (not part of the step): the other
-    causal shapes, prefill 3 on (batch, sequence, heads, dim) tensors (fa_fwd_bshd), sliding
-    window (6, 8), chunked prefill (7, 8), paged decode (9) and FP8 decode (10).  Caches of
-    decode 9 and 10 (over 1 GB) exceed L2; prefill 1 does not."""
+def _time_calls(run, n: int, stream) -> float:
+    """Mean milliseconds per call of run() over n calls after 3 warm-up calls, from CUDA
+    events recorded on the stream the kernels are launched on."""
+    for _ in range(3):
+        run()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    torch.cuda.synchronize()
+    e[0].record(stream)
+    for _ in range(n):
+        run()
+    e[1].record(stream)
+    torch.cuda.synchronize()
+    return e[0].elapsed_time(e[1]) / n
+
+
+def run_configs(dev, peaks, world):
+    """Kernel times for every other named workload, one library call per timed iteration:
+    prefill 1 (small, fp32 output: launch-bound), the grouped-query causal prefills 3 (also
+    on (batch, sequence, heads, dim) tensors through fa_fwd_bshd) and 4, sliding window (6, 8),
+    chunked prefill (7, 8), paged decode (9) and FP8 decode (10).  Every input but prefill 1's
+    exceeds the 126 MB L2, so back-to-back calls do not hit in L2.  Times are the max over
+    ranks; throughputs are per GPU."""
     from exact_io_aware_81_b200 import ops
-    res = {}
+    tensor_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    stream = torch.cuda.current_stream(dev)
+    res, launches = {}, 0
     for kid, bshd in ((1, False), (3, False), (3, True), (4, False), (6, False), (7, False), (8, False)):
         w = inputs.workload(kid)
         B, Hq, Hkv, Nq, Nk, d = w.shape
@@ -444,20 +494,28 @@ def run_extra(args, dev, peaks):
             q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
             o = torch.empty((B, Hq, Nq, d), dtype=w.out_dtype, device=dev)
             fwd = ops.fwd
-        n = 3 if kid != 1 else 20
-        for _ in range(3):
-            fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse, window=w.window)
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        e[0].record()
-        for _ in range(n):
-            fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse, window=w.window)
-        e[1].record()
-        torch.cuda.synchronize(dev)
-        ms = e[0].elapsed_time(e[1]) / n
+        n = 50 if kid == 1 else 10
+        ms = _time_calls(lambda: fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o,
+                                     lse=lse, window=w.window, stream=stream), n, stream)
+        launches += n
+        ms = max_over_ranks(ms, world, dev)
         tf = w.flops() / (ms * 1e-3) / 1e12
-        res[w.name + ("_bshd" if bshd else "")] = {"ms": ms, "tflops": tf,
-                                                   "frac": tf / peaks.get("bf16_tflops", 1590.0)}
-        del q, k, v, o, lse
+        entry = {"workload": w.name + ("_bshd" if bshd else ""), "ms": ms, "tflops": tf,
+                 "frac": tf / tensor_peak, "bound": "tensor", "algorithmic_flops": w.flops(),
+                 "kernel": PREFILL_KERNEL}
+        if kid == 1:
+            # host cost of one call (binding, C ABI, cached tensor maps, launch), wall clock;
+            # the calls only enqueue, and the queue does not fill in 200 calls
+            torch.cuda.synchronize()
+            t = time.perf_counter()
+            for _ in range(200):
+                fwd(q, k, v, causal=w.causal, scale=w.scale, out_dtype=w.out_dtype, out=o, lse=lse,
+                    window=w.window, stream=stream)
+            entry["host_us_per_call"] = (time.perf_counter() - t) / 200 * 1e6
+            torch.cuda.synchronize()
+            launches += 200
+        res[f"workload{kid}" + ("_bshd" if bshd else "")] = entry
+        del q, k, v, o, lse, w
         torch.cuda.empty_cache()
     # decode over a paged cache (9) and over an FP8 cache (10): HBM-bound like decode 5
     for kid in (9, 10):
@@ -471,28 +529,26 @@ def run_extra(args, dev, peaks):
             kp, vp, bt = w.kpages.to(dev), w.vpages.to(dev), w.block_table.to(dev)
             nmax = kp.shape[2] * bt.shape[1]
             wsp = torch.empty(ops.decode_workspace_size(B, Hq, nmax, d), dtype=torch.uint8, device=dev)
-            run = lambda: ops.decode_paged(qd, kp, vp, bt, sl, scale=w.scale, workspace=wsp, out=out, lse=ls)
+            run = lambda: ops.decode_paged(qd, kp, vp, bt, sl, scale=w.scale, workspace=wsp, out=out, lse=ls,
+                                           stream=stream)
+            kern = "fa_decode_split_kernel (paged) + fa_decode_merge_kernel"
         else:
             kc, vc = w.kcache.to(dev), w.vcache.to(dev)
             ks, vs = w.k_scale.to(dev), w.v_scale.to(dev)
             wsp = torch.empty(ops.decode_workspace_size(B, Hq, kc.shape[2], d), dtype=torch.uint8, device=dev)
-            run = lambda: ops.decode_fp8(qd, kc, vc, ks, vs, sl, scale=w.scale, workspace=wsp, out=out, lse=ls)
-        for _ in range(3):
-            run()
+            run = lambda: ops.decode_fp8(qd, kc, vc, ks, vs, sl, scale=w.scale, workspace=wsp, out=out, lse=ls,
+                                         stream=stream)
+            kern = "fa_decode_fp8_kernel + fa_decode_merge_kernel"
         n = 20
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        e[0].record()
-        for _ in range(n):
-            run()
-        e[1].record()
-        torch.cuda.synchronize(dev)
-        ms = e[0].elapsed_time(e[1]) / n
+        ms = max_over_ranks(_time_calls(run, n, stream), world, dev)
+        launches += 2 * n
         gbs = w.io_bytes() / (ms * 1e-3) / 1e9
-        res[w.name] = {"ms": ms, "gbs": gbs, "frac": gbs / peaks.get("hbm_gbs", 6650.0),
-                       "cache_bytes": w.cache_bytes()}
+        res[f"workload{kid}"] = {"workload": w.name, "ms": ms, "gbs": gbs, "frac": gbs / hbm_peak, "bound": "hbm",
+                                 "algorithmic_bytes": w.io_bytes(), "kernel": kern}
         del w, run
         torch.cuda.empty_cache()
     assert ops.get_error() == ops.FA_OK
+    res["_launches"] = launches
     return res
 
 
@@ -503,14 +559,20 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-s", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-step-s", type=float, default=0.5, help="seconds per reference-arm step")
-    ap.add_argument("--extra", action="store_true", help="also time the other prefill workloads")
+    ap.add_argument("--no-configs", action="store_true", help="skip timing the other named workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: start the ranks, and pass on their exit status
+        import subprocess
+        raise SystemExit(subprocess.call(relaunch_cmd(args.gpus, sys.argv[1:], free_port())))
     rank, world, local = dist_setup(args)
     if args.impl == "reference":
         if rank == 0:  # under torchrun the other ranks exit without work

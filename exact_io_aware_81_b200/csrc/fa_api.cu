@@ -99,25 +99,75 @@ EncodeTiledFn get_encode_fn()
     return fn;
 }
 
+// Encoded maps are cached on the host, keyed by every argument of the encode call (data
+// type, rank, base address, sizes, strides, box): a map is a pure function of these, so a
+// hit returns exactly what re-encoding would.  Repeated calls on the same buffers (a
+// serving loop, a benchmark) then skip the driver's encode, about a microsecond per map.
+struct MapKey {
+    int dtype, rank;
+    const void *base;
+    cuuint64_t dims[4], strides[3];
+    cuuint32_t box[4];
+};
+constexpr int kMapCacheSize = 64;
+struct MapCache {
+    MapKey key[kMapCacheSize];
+    CUtensorMap map[kMapCacheSize];
+    bool used[kMapCacheSize] = {};
+    int next = 0;
+};
+MapCache g_maps;
+std::mutex g_maps_mu;
+
+int encode_map_cached(CUtensorMap *m, CUtensorMapDataType dtype, int rank, const void *base,
+                      const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box)
+{
+    MapKey k;
+    memset(&k, 0, sizeof k);  // padding too: keys are compared bytewise
+    k.dtype = (int)dtype;
+    k.rank = rank;
+    k.base = base;
+    for (int i = 0; i < rank; ++i) {
+        k.dims[i] = dims[i];
+        k.box[i] = box[i];
+        if (i + 1 < rank) k.strides[i] = strides[i];
+    }
+    {
+        std::lock_guard<std::mutex> lk(g_maps_mu);
+        for (int i = 0; i < kMapCacheSize; ++i)
+            if (g_maps.used[i] && memcmp(&g_maps.key[i], &k, sizeof k) == 0) {
+                *m = g_maps.map[i];
+                return FA_OK;
+            }
+    }
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, dtype, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    std::lock_guard<std::mutex> lk(g_maps_mu);
+    const int slot = g_maps.next;
+    g_maps.next = (slot + 1) % kMapCacheSize;
+    g_maps.key[slot] = k;
+    g_maps.map[slot] = *m;
+    g_maps.used[slot] = true;
+    return FA_OK;
+}
+
 // A (D, rows, planes) bf16 tensor with boxes of `box_rows` rows x 64 columns, 128-byte
 // swizzle.
 int encode_rows_map(CUtensorMap *m, const void *base, int D, long long rows, long long planes,
                     unsigned box_rows = 128, bool fp8 = false)
 {
-    EncodeTiledFn fn = get_encode_fn();
-    if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     // one box row is 128 bytes: 64 bf16 or 128 FP8 (byte) elements
     const cuuint64_t eb = fp8 ? 1 : 2;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
-    cuuint64_t strides[2] = {(cuuint64_t)D * eb, (cuuint64_t)rows * D * eb};
-    cuuint32_t box[3] = {(cuuint32_t)(128 / eb), box_rows, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                    const_cast<void *>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-    return FA_OK;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * eb, (cuuint64_t)rows * D * eb};
+    const cuuint32_t box[3] = {(cuuint32_t)(128 / eb), box_rows, 1};
+    return encode_map_cached(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base,
+                             dims, strides, box);
 }
 
 // A prefill operand as a 4-D (d, rows, heads, batch) bf16 tensor with boxes of `box_rows`
@@ -126,18 +176,11 @@ int encode_rows_map(CUtensorMap *m, const void *base, int D, long long rows, lon
 int encode_heads_map(CUtensorMap *m, const void *base, int D, int rows, int heads, int batch, bool bshd,
                      unsigned box_rows = 128)
 {
-    EncodeTiledFn fn = get_encode_fn();
-    if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const cuuint64_t row = (cuuint64_t)D * 2, plane = (cuuint64_t)rows * heads * row;
-    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)batch};
-    cuuint64_t strides[3] = {bshd ? heads * row : row, bshd ? row : rows * row, plane};
-    cuuint32_t box[4] = {64, box_rows, 1, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-    return FA_OK;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)batch};
+    const cuuint64_t strides[3] = {bshd ? heads * row : row, bshd ? row : rows * row, plane};
+    const cuuint32_t box[4] = {64, box_rows, 1, 1};
+    return encode_map_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box);
 }
 
 // ------------------------------------------------------------------- prefill
@@ -348,7 +391,7 @@ struct CacheDesc {
 // length (ignored when paged: page_size * max_pages).
 int decode_general(const void *q, const CacheDesc &c, const int *seqlens, void *o, float *lse,
                    int B, int Hq, int Hkv, int Nmax, int d, float scale, void *workspace,
-                   size_t workspace_bytes, void *stream, int o_dtype = FA_BF16)
+                   size_t workspace_bytes, void *stream, int o_dtype = FA_BF16, int selftest = 0)
 {
     if (o_dtype != FA_BF16 && o_dtype != FA_F32) return fail(FA_ERR_INVALID, "unknown output dtype %d", o_dtype);
     if (!q || !c.k || !c.v || !seqlens || !o) return fail(FA_ERR_INVALID, "null pointer argument");
@@ -424,6 +467,7 @@ int decode_general(const void *q, const CacheDesc &c, const int *seqlens, void *
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     p.wait_limit_ns = g_wait_limit_ns;
+    p.selftest_no_full = selftest;
     if (c.fp8)
         rc = c.paged ? launch_split_rg<128, true, true>(p, rg, info, st) : launch_split_rg<128, false, true>(p, rg, info, st);
     else if (c.paged)
@@ -505,6 +549,19 @@ int fa_decode_ex(const void *q, const void *kcache, const void *vcache, const in
                           stream, o_dtype);
 }
 
+int fa_decode_selftest_timeout(const void *q, const void *kcache, const void *vcache, const float *k_scale,
+                               const float *v_scale, const int *seqlens, void *o, float *lse, int B, int Hq,
+                               int Hkv, int Nmax, int d, float scale, void *workspace, size_t workspace_bytes,
+                               void *stream)
+{
+    if ((k_scale == nullptr) != (v_scale == nullptr))
+        return fail(FA_ERR_INVALID, "give both FP8 scale pointers or neither");
+    const bool fp8 = k_scale != nullptr;
+    const CacheDesc c{kcache, vcache, fp8, k_scale, v_scale, false, nullptr, 0, 0, 0};
+    return decode_general(q, c, seqlens, o, lse, B, Hq, Hkv, Nmax, d, scale, workspace, workspace_bytes,
+                          stream, FA_BF16, 1);
+}
+
 int fa_merge_lse(const float *o_parts, const float *lse_parts, int P, int rows, int d, void *o,
                  float *lse, int o_dtype, void *stream)
 {
@@ -557,27 +614,62 @@ int fa_decode_paged_fp8(const void *q, const void *kpages, const void *vpages, c
 // For callers that cannot allocate device memory (see fa_decode_noalloc in fa.h): the
 // split-KV partials live in this fixed array instead of a caller workspace.  In host code
 // `g_noalloc_scratch` only names a host-side stand-in; its device address is looked up
-// once per device with cudaGetSymbolAddress and that address is what the kernels get.
+// with cudaGetSymbolAddress, with the device current, and that address is what the kernels
+// get.  The lookup is done on a device's first call and again whenever the device's
+// context has changed since (a cudaDeviceReset unloads the module and the array with it).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
-void *g_noalloc_ptr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context (0 if it cannot be read).
+unsigned long long current_context_id()
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+struct NoallocScratch {
+    void *ptr = nullptr;
+    unsigned long long ctx_id = 0;
+};
+NoallocScratch g_noalloc[kMaxDevices];
 std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on the current device (looked up on first use).
+// Device address of the scratch array on the current device, in its current context.
 int noalloc_scratch(int dev, void **out)
 {
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    NoallocScratch &c = g_noalloc[dev];
+    if (!c.ptr || ctx == 0 || ctx != c.ctx_id) {
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || !p)
             return fail(FA_ERR_CUDA, "cudaGetSymbolAddress of the decode scratch: %s",
                         cudaGetErrorString(e));
-        g_noalloc_ptr[dev] = p;
+        c.ptr = p;
+        c.ctx_id = ctx;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = c.ptr;
     return FA_OK;
 }
 

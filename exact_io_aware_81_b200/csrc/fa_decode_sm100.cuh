@@ -83,6 +83,9 @@ struct DecodeParams {
     const int *block_table;   // (B, max_pages) physical page of each logical page
     int page_size, max_pages, num_pages;
     int box_rows;             // rows per copy: a power of two <= 64 that divides page_size
+    // time-limit self-test: the producer of every CTA withholds its first copy (neither the
+    // arrive nor the copy is issued), so the consumers' first wait must run out
+    int selftest_no_full;
 };
 
 namespace decode {
@@ -311,7 +314,9 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                     const uint32_t st = ring % C::kStages;
                     const uint32_t ph = (ring / C::kStages) & 1u;
                     if (!wait_warp(&empty[st], ph ^ 1u, sf)) { ok = false; break; }
-                    if (PAGED) {
+                    if (p.selftest_no_full && ring == 0) {
+                        // self-test: this stage is never filled (see DecodeParams)
+                    } else if (PAGED) {
                         // only the boxes that hold keys of the sequence are copied (rows past
                         // it are masked or cleared by the consumers)
                         const int nbox = (min(kSub, n - t * kSub) + p.box_rows - 1) / p.box_rows;
@@ -344,6 +349,7 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
         if (leader) {
             for (uint32_t st = 0; st < (uint32_t)C::kStages && st < ring; ++st) {
                 const uint32_t last = ring - 1 - ((ring - 1 - st) % C::kStages);
+                if (p.selftest_no_full && last == 0) continue;  // never issued
                 const uint32_t par = (last / C::kStages) & 1u;
                 const uint64_t t0 = ptx::globaltimer_ns();
                 while (!ptx::mbar_test(&full[st], par))
@@ -647,7 +653,9 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                 uint64_t *fb = &full[2 * w + v];
                 const CUtensorMap *map = v ? &p.tm_v : &p.tm_k;
                 const int key0 = start[w] + (s[w] >> 1) * SK;
-                if (PAGED) {
+                if (p.selftest_no_full && w == 0 && v == 0 && f == 0u) {
+                    // self-test: worker 0's first K block is never filled (see DecodeParams)
+                } else if (PAGED) {
                     // only the boxes that hold keys of the sequence are copied (rows past it
                     // are masked or cleared by the worker)
                     const int nbox = (min(SK, start[w] + n[w] - key0) + p.box_rows - 1) / p.box_rows;
@@ -703,7 +711,8 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
 #pragma unroll
                 for (int v = 0; v < 2; ++v) {
                     const uint32_t f = v ? vfill[w] : kfill[w];
-                    if (f > 0u) {
+                    const bool withheld = p.selftest_no_full && w == 0 && v == 0 && f == 1u;
+                    if (f > 0u && !withheld) {
                         const uint64_t t0 = ptx::globaltimer_ns();
                         while (!ptx::mbar_test(&full[2 * w + v], (f - 1u) & 1u))
                             if (ptx::globaltimer_ns() - t0 > p.wait_limit_ns) { raise_error(kErrTimeout); break; }

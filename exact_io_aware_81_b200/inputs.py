@@ -376,8 +376,14 @@ def workload(k: int):
     raise KeyError(k)
 
 
-def sample_rows(N: int, count: int, seed: int, tile: int = 128) -> torch.Tensor:
-    """Seeded sorted row sample that always holds 0, 1, N-1 and the tile edges (t*tile-1, t*tile)."""
+def sample_rows(N: int, interior: int, seed: int, tile: int = 128) -> torch.Tensor:
+    """Seeded sorted row sample: the fixed rows 0, 1, N-1 and both edges of every tile
+    boundary (t*tile - 1, t*tile), plus ``interior`` further rows drawn at random, without
+    replacement, from the rows not already fixed (all of them if fewer remain).
+
+    With 128-row tiles the fixed rows are tensor-memory lanes 0, 1 and 127 of a tile; the
+    random rows land on every other lane, so a sample checks the rows of every softmax warp.
+    """
     fixed = {0, 1, N - 1}
     for t in range(1, (N + tile - 1) // tile):
         fixed.add(t * tile - 1)
@@ -385,11 +391,12 @@ def sample_rows(N: int, count: int, seed: int, tile: int = 128) -> torch.Tensor:
     fixed = {r for r in fixed if 0 <= r < N}
     gen = torch.Generator("cpu")
     gen.manual_seed(seed)
-    extra = max(0, count - len(fixed))
-    perm = torch.randperm(N, generator=gen)[: extra + len(fixed)].tolist()
     rows = set(fixed)
-    for r in perm:
-        if len(rows) >= max(count, len(fixed)):
+    added = 0
+    for r in torch.randperm(N, generator=gen).tolist():
+        if added >= interior:
             break
-        rows.add(r)
+        if r not in fixed:
+            rows.add(r)
+            added += 1
     return torch.tensor(sorted(rows), dtype=torch.int32)

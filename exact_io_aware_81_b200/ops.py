@@ -48,6 +48,7 @@ SIGNATURES = {
     "fa_get_error": (_I, [_P]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "fa_fwd_selftest_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_decode_selftest_timeout": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_status_str": (ctypes.c_char_p, [_I]),
     "fa_last_error_message": (ctypes.c_char_p, []),
     "fa_version": (_I, []),
@@ -455,6 +456,27 @@ def fwd_selftest_timeout(q, k, v, causal=False, scale=None, stream=None):
         rc = load().fa_fwd_selftest_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                             lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
                                             int(bool(causal)), _stream_handle(stream, dev))
+    _check(rc)
+    return out, lse
+
+
+def decode_selftest_timeout(q, kcache, vcache, seqlens, k_scale=None, v_scale=None, scale=None, stream=None):
+    """Run a decode (bf16 caches, or E4M3 caches when both scales are given) with the split
+    kernel's first copy withheld in every CTA (time-limit self-test)."""
+    B, Hq, d = q.shape
+    Hkv, Nmax = kcache.shape[1], kcache.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws = torch.empty(decode_workspace_size(B, Hq, Nmax, d), dtype=torch.uint8, device=q.device)
+    with _on_device(q, kcache, vcache, seqlens, out, lse, ws, k_scale, v_scale) as dev:
+        rc = load().fa_decode_selftest_timeout(
+            q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
+            k_scale.data_ptr() if k_scale is not None else None,
+            v_scale.data_ptr() if v_scale is not None else None, seqlens.data_ptr(), out.data_ptr(),
+            lse.data_ptr(), B, Hq, Hkv, Nmax, d, float(scale), ws.data_ptr(), ws.numel(),
+            _stream_handle(stream, dev))
     _check(rc)
     return out, lse
 

@@ -232,7 +232,8 @@ FA_API int fa_decode_paged_fp8(const void *q, const void *kpages, const void *vp
  *     larger problems are rejected with FA_ERR_WORKSPACE and nothing is launched.
  *   - The first call on each device looks up the device address of the scratch array
  *     (cudaGetSymbolAddress) with that device current; make that first call before any
- *     stream capture begins.
+ *     stream capture begins.  The lookup is repeated when the device's context has
+ *     changed since (after a cudaDeviceReset, whose module reload moves the array).
  *   - Every call, on every stream, shares the one scratch array and leaves its contents
  *     behind.  Nothing in it needs to start at zero (each call writes every partial it
  *     reads), but calls whose kernels overlap on the GPU race on it: order them (one
@@ -267,6 +268,21 @@ FA_API void fa_set_wait_limit_ns(unsigned long long ns);
 FA_API int fa_fwd_selftest_timeout(const void *q, const void *k, const void *v, void *o, float *lse,
                             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
                             int causal, void *stream);
+
+/*
+ * Self-test of the time-limit path of the decode kernels: runs the decode of fa_decode
+ * (k_scale = v_scale = NULL: bf16 caches) or of fa_decode_fp8 (both scales given: E4M3
+ * caches) on the given (valid) arguments, with the producer warp of every split-kernel CTA
+ * withholding its first copy, so that the consumers' first wait must run out after the
+ * wait limit; the merge kernel that follows runs on whatever the partials hold.  The
+ * outputs are left unspecified; fa_get_error afterwards returns FA_ERR_TIMEOUT.  Nothing
+ * faults or hangs: every wait is bounded and every copy that was issued lands before the
+ * kernel exits.
+ */
+FA_API int fa_decode_selftest_timeout(const void *q, const void *kcache, const void *vcache,
+                                      const float *k_scale, const float *v_scale, const int *seqlens,
+                                      void *o, float *lse, int B, int Hq, int Hkv, int Nmax, int d,
+                                      float scale, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 FA_API const char *fa_status_str(int status);

@@ -101,3 +101,42 @@ def test_reference_arm_runs_on_cpu():
     assert out["config"] == bench.step_config(1) and out["steps"] == 1 and out["warmup"] == 3
     assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["value"] == out["value"]
     assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["e2e"]["value"] == out["value"]
+
+
+def _env_without_ranks():
+    env = dict(os.environ)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT", "LOCAL_WORLD_SIZE"):
+        env.pop(k, None)
+    return env
+
+
+@pytest.mark.slow
+def test_gpus_option_starts_one_rank_per_gpu():
+    """`bench.py --gpus 2` started without torchrun re-launches itself as two ranks; the
+    reference arm (CPU only) lets this run here: rank 0 prints the one line, with n_gpus 2."""
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
+                        "--warmup", "3", "--ref-step-s", "0.05"], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600, env=_env_without_ranks())
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and out["n_gpus"] == 2
+    assert out["config"] == bench.step_config(2)
+
+
+def test_relaunch_command_is_torchrun_on_loopback():
+    cmd = bench.relaunch_cmd(4, ["--gpus", "4", "--steps", "5"], 12345)
+    assert cmd[:3] == [sys.executable, "-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-port=12345" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "5"] and cmd[-5].endswith("bench.py")
+
+
+def test_world_size_must_match_gpus():
+    env = _env_without_ranks()
+    env.update(WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "1", "--steps", "1",
+                        "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode != 0
+    assert "--gpus 1 but WORLD_SIZE=2" in r.stderr

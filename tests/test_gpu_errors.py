@@ -1,9 +1,12 @@
 """Device-side error reporting, without faulting, trapping or hanging the GPU.
 
-The time-limit test withholds one internal signal (the score-ready arrive of the MMA
-warp), so the softmax warps' bounded wait runs out after a short limit; the kernel must
-record FA_ERR_TIMEOUT, stop every role at its next wait, free its tensor memory and
-return, leaving the context usable for the normal call that follows.
+Each time-limit test withholds one internal signal so that a bounded wait runs out after a
+short limit: in the prefill kernel the score-ready arrive of the MMA warp, in the decode
+split kernels (bf16 shared ring, FP8 per-warp rings) the first copy of every CTA's producer.
+The kernel must record FA_ERR_TIMEOUT, stop every role at its next wait, let the copies
+already issued land, free its tensor memory and return; for decode the merge kernel, a
+programmatic dependent of the split kernel, then still runs and ends.  The context must stay
+usable: a normal call right after matches the oracle.
 """
 import pytest
 import torch
@@ -30,3 +33,37 @@ def test_wait_limit_expires_cleanly():
     assert ops.get_error() == ops.FA_OK
     ro, rl = oracle.attn_fwd(w.q, w.k, w.v, w.scale, True)
     compare(o, lse, ro, rl, "after timeout")
+
+
+@pytest.mark.parametrize("Hq,Hkv,d", [(8, 2, 128), (6, 6, 64)])
+def test_decode_wait_limit_expires_cleanly(Hq, Hkv, d):
+    w = inputs.make_decode(5, Hq, Hkv, 1500, d, seed=13, len_range=(1, 1500))
+    q, kc, vc, sl = w.q.cuda(), w.kcache.cuda(), w.vcache.cuda(), w.seqlens.cuda()
+    ops.set_wait_limit_ns(20_000_000)
+    try:
+        ops.decode_selftest_timeout(q, kc, vc, sl, scale=w.scale)
+        assert ops.get_error() == ops.FA_ERR_TIMEOUT
+        assert ops.get_error() == ops.FA_OK
+    finally:
+        ops.set_wait_limit_ns(0)
+    o, lse = ops.decode(q, kc, vc, sl, scale=w.scale)
+    assert ops.get_error() == ops.FA_OK
+    compare(o, lse, *oracle.decode(w.q, w.kcache, w.vcache, w.seqlens, w.scale), "decode after timeout")
+
+
+def test_fp8_decode_wait_limit_expires_cleanly():
+    w = inputs.make_fp8_decode(5, 8, 2, 1500, 128, seed=14, len_range=(1, 1500))
+    args = [t.cuda() for t in (w.q, w.kcache, w.vcache, w.seqlens)]
+    ks, vs = w.k_scale.cuda(), w.v_scale.cuda()
+    ops.set_wait_limit_ns(20_000_000)
+    try:
+        ops.decode_selftest_timeout(*args, k_scale=ks, v_scale=vs, scale=w.scale)
+        assert ops.get_error() == ops.FA_ERR_TIMEOUT
+        assert ops.get_error() == ops.FA_OK
+    finally:
+        ops.set_wait_limit_ns(0)
+    q, kc, vc, sl = args
+    o, lse = ops.decode_fp8(q, kc, vc, ks, vs, sl, scale=w.scale)
+    assert ops.get_error() == ops.FA_OK
+    compare(o, lse, *oracle.decode_fp8(w.q, w.kcache, w.vcache, w.k_scale, w.v_scale, w.seqlens, w.scale),
+            "FP8 decode after timeout")

@@ -3,8 +3,9 @@
 Small problems are compared in full; they span several 128-row tiles, ragged tails, the
 GQA / MQA / MHA head mappings (and an odd group size), d = 64 and 128, causal and not,
 Nq < Nk causal, and N = 1.  The named full-size workloads run in the benchmark's launch
-configuration and are compared on seeded row samples that always hold the first and last
-rows and the tile edges.  Outputs are written into guarded buffers whose NaN guard bands
+configuration: workload 2 on every row, the long grouped-query workloads on 256 random
+rows per (b, h) on top of the first, last and tile-edge rows, so that every softmax
+warp's rows are compared.  Outputs are written into guarded buffers whose NaN guard bands
 must stay untouched.
 """
 import math
@@ -74,15 +75,35 @@ def test_workload1_full(out_dtype):
     compare(o, lse, ro, rl, "workload 1")
 
 
-@pytest.mark.parametrize("k,rows_per_head", [(2, 48), (3, 16), (4, 8)])
-def test_named_workload_sampled(k, rows_per_head):
+def test_workload2_full():
+    """The causal MHA workload, every row of every (b, h) against the oracle."""
+    w = inputs.workload(2)
+    o, lse = run_gpu(w)
+    ro, rl = oracle.attn_fwd(w.q, w.k, w.v, w.scale, w.causal)
+    compare(o, lse, ro, rl, "workload 2 (all rows)")
+
+
+def interior_lanes(rows: torch.Tensor) -> dict:
+    """How many sampled rows fall on each 32-lane quarter of a 128-row tile, edge lanes
+    0, 1 and 127 left out: every softmax warp must have rows in the comparison."""
+    lanes = rows.long() % 128
+    inner = lanes[(lanes >= 2) & (lanes <= 126)]
+    return {qtr: int(((inner // 32) == qtr).sum()) for qtr in range(4)}
+
+
+@pytest.mark.parametrize("k,interior", [(3, 256), (4, 256)])
+def test_named_workload_sampled(k, interior):
+    """The long GQA workloads on 256 random rows per (b, h) on top of the first, last and
+    tile-edge rows."""
     w = inputs.workload(k)
     B, Hq, Hkv, Nq, Nk, d = w.shape
     o, lse = run_gpu(w)
-    rows = inputs.sample_rows(Nq, rows_per_head, seed=77 + k)
+    rows = inputs.sample_rows(Nq, interior, seed=77 + k)
+    assert min(interior_lanes(rows).values()) >= 32, interior_lanes(rows)
     ro, rl = oracle.attn_fwd(w.q, w.k, w.v, w.scale, w.causal, rows=rows)
     idx = rows.long().to(DEV)
-    compare(o.index_select(2, idx), lse.index_select(2, idx), ro, rl, f"workload {k}")
+    compare(o.index_select(2, idx), lse.index_select(2, idx), ro, rl,
+            f"workload {k} ({len(rows)} rows per head, interior lanes {interior_lanes(rows)})")
     # properties at full size: every LSE finite and every O row a convex combination of V
     assert torch.isfinite(lse).all()
     assert torch.isfinite(o.float()).all()
