@@ -205,6 +205,82 @@ def make_fp8_decode(B: int, Hq: int, Hkv: int, Nmax: int, d: int, *, seed: int,
                      v_scale=vs, seqlens=seqlens, scale=float(scale))
 
 
+@dataclasses.dataclass
+class Fp8Prefill:
+    """One prefill problem over FP8 E4M3 tensors: q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d) uint8
+    bytes; q_scale (Hq,), k_scale/v_scale (Hkv,) float32.  Row i of query head h is
+    q_scale[h] * e4m3(q[b, h, i, :]); likewise K and V with their head's scale."""
+    name: str
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    q_scale: torch.Tensor
+    k_scale: torch.Tensor
+    v_scale: torch.Tensor
+    causal: bool
+    scale: float
+    window: int = 0
+    out_dtype: torch.dtype = torch.bfloat16
+
+    @property
+    def shape(self):
+        B, Hq, Nq, d = self.q.shape
+        Hkv, Nk = self.k.shape[1], self.k.shape[2]
+        return B, Hq, Hkv, Nq, Nk, d
+
+    def pairs(self) -> int:
+        B, Hq, Hkv, Nq, Nk, d = self.shape
+        return B * Hq * allowed_pairs(Nq, Nk, self.causal, self.window)
+
+    def flops(self) -> float:
+        """Algorithmic flops: 2*d for q.k plus 2*d for p*v, per allowed pair."""
+        return 4.0 * self.shape[5] * self.pairs()
+
+    def io_bytes(self) -> int:
+        """Read the E4M3 Q, K, V and the scales, write O and LSE."""
+        B, Hq, Hkv, Nq, Nk, d = self.shape
+        ob = 4 if self.out_dtype == torch.float32 else 2
+        return (B * Hq * Nq * d + 2 * B * Hkv * Nk * d) + ob * B * Hq * Nq * d + 4 * B * Hq * Nq + 4 * (Hq + 2 * Hkv)
+
+
+def make_fp8_prefill(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, *, seed: int,
+                     causal: bool, window: int = 0, scale: Optional[float] = None,
+                     head_std_range: Optional[tuple] = (0.5, 2.0),
+                     outlier_rows_frac: float = 0.0, outlier_factor: float = 3.0,
+                     name: str = "fp8_prefill") -> Fp8Prefill:
+    """Draw a seeded prefill problem and encode it in FP8 E4M3 with one scale per head.
+
+    Draw order: per-head standard deviations (Q heads, then K heads, then V heads, uniform
+    in head_std_range) -> Q -> K -> V (fp32) -> outlier key rows (as make_prefill); then
+    each tensor is encoded per head with quantize_e4m3.
+    """
+    assert Hq % Hkv == 0
+    gen = torch.Generator("cpu")
+    gen.manual_seed(seed)
+    q_std = k_std = v_std = None
+    if head_std_range is not None:
+        lo, hi = head_std_range
+        q_std = (lo + (hi - lo) * torch.rand((Hq,), generator=gen)).view(1, Hq, 1, 1)
+        k_std = (lo + (hi - lo) * torch.rand((Hkv,), generator=gen)).view(1, Hkv, 1, 1)
+        v_std = (lo + (hi - lo) * torch.rand((Hkv,), generator=gen)).view(1, Hkv, 1, 1)
+    q = _randn(gen, (B, Hq, Nq, d), q_std)
+    k = _randn(gen, (B, Hkv, Nk, d), k_std)
+    v = _randn(gen, (B, Hkv, Nk, d), v_std)
+    if outlier_rows_frac > 0.0:
+        n_out = int(round(outlier_rows_frac * Nk))
+        for b in range(B):
+            for g in range(Hkv):
+                rows = torch.randperm(Nk, generator=gen)[:n_out]
+                k[b, g, rows, :] *= outlier_factor
+    q8, qs = quantize_e4m3(q)
+    k8, ks = quantize_e4m3(k)
+    v8, vs = quantize_e4m3(v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    return Fp8Prefill(name=name, q=q8, k=k8, v=v8, q_scale=qs, k_scale=ks, v_scale=vs, causal=causal,
+                      scale=float(scale), window=int(window))
+
+
 def allowed_pairs(Nq: int, Nk: int, causal: bool, window: int = 0) -> int:
     """Pairs (i, j) with key j visible to query i.
 
@@ -340,11 +416,15 @@ WORKLOADS = {
     9: "gqa_paged_decode_b32_hq32_hkv8_page64_nmax8192_d128",
     # decode 5 over an FP8 (E4M3) cache with per-head scales (youngju.dev sections 5, 7)
     10: "gqa_fp8kv_decode_b32_hq32_hkv8_nmax8192_d128",
+    # prefill over FP8 (E4M3) Q, K, V with per-head scales (toolsku.com, FlashAttention
+    # generations table: FP8 among FA3's data types): workloads 2 and 3 encoded in FP8
+    11: "fp8_mha_causal_prefill_b8_h32_n2048_d128",
+    12: "fp8_gqa_causal_prefill_b4_hq32_hkv8_n8192_d128",
 }
 
 
 def workload(k: int):
-    """Return workload k (1..5) with seed 1000+k."""
+    """Return named workload k (see WORKLOADS) drawn with seed 1000+k."""
     seed = 1000 + k
     name = WORKLOADS[k]
     if k == 1:
@@ -373,6 +453,11 @@ def workload(k: int):
                                  name=name)
     if k == 10:
         return make_fp8_decode(32, 32, 8, 8192, 128, seed=seed, len_range=(1024, 8192), name=name)
+    if k == 11:
+        return make_fp8_prefill(8, 32, 32, 2048, 2048, 128, seed=seed, causal=True, head_std_range=None,
+                                outlier_rows_frac=0.01, outlier_factor=3.0, name=name)
+    if k == 12:
+        return make_fp8_prefill(4, 32, 8, 8192, 8192, 128, seed=seed, causal=True, name=name)
     raise KeyError(k)
 
 

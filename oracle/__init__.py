@@ -5,7 +5,8 @@ may import this package.  It shares no code with the CUDA path (``exact_io_aware
 and never imports it; the two meet only through the seeded inputs.
 
 Contents:
-  * ``attn_fwd`` / ``decode`` / ``decode_paged`` / ``decode_fp8`` / ``probs``: the fp64
+  * ``attn_fwd`` / ``attn_fwd_fp8`` / ``decode`` / ``decode_paged`` / ``decode_fp8`` /
+    ``probs``: the fp64
     two-pass definition, in plain C with OpenMP (``attn_oracle.c``), called through
     ctypes; ``e4m3_to_double`` decodes one FP8 E4M3 byte.
   * ``online.online_attention``: a restatement of the block-by-block online softmax
@@ -54,12 +55,13 @@ def declare(lib):
     lib.oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, D, P, P]
     lib.oracle_decode_paged.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, P]
     lib.oracle_decode_fp8.argtypes = [P, P, P, P, P, P, I, I, I, I, I, D, P, P]
+    lib.oracle_attn_fwd_fp8.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, D, I, I, P, I, P, P]
     lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
     lib.oracle_e4m3_to_double.restype = D
     lib.oracle_num_threads.argtypes = []
     for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_window, lib.oracle_attn_probs,
               lib.oracle_attn_probs_window, lib.oracle_decode, lib.oracle_decode_paged,
-              lib.oracle_decode_fp8, lib.oracle_num_threads):
+              lib.oracle_decode_fp8, lib.oracle_attn_fwd_fp8, lib.oracle_num_threads):
         f.restype = I
     return lib
 
@@ -197,4 +199,33 @@ def decode_fp8(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor,
                                    B, Hq, Hkv, Nmax, d, float(scale), _ptr(o), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_decode_fp8 rejected its arguments")
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def attn_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_scale: torch.Tensor,
+                 k_scale: torch.Tensor, v_scale: torch.Tensor, scale: float, causal: bool,
+                 rows: Optional[torch.Tensor] = None, window: int = 0):
+    """fp64 attention of FP8 E4M3 q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d) (uint8 bytes) with
+    per-head dequantization scales: q row of head h is q_scale[h] * e4m3(bytes), K and V
+    rows of head g are k_scale[g] * e4m3 and v_scale[g] * e4m3.  Rows and window as in
+    attn_fwd; returns (o, lse) float64."""
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    for t in (q, k, v):
+        assert t.dtype == torch.uint8, t.dtype
+    qb, kb, vb = (np.ascontiguousarray(t.detach().cpu().numpy()) for t in (q, k, v))
+    qs, ks, vs = (np.ascontiguousarray(t.detach().cpu().numpy().astype(np.float32))
+                  for t in (q_scale, k_scale, v_scale))
+    if rows is not None:
+        rw = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+        nr, rp = int(rw.shape[0]), _ptr(rw)
+    else:
+        rw, nr, rp = None, Nq, None
+    o = np.empty((B, Hq, nr, d), dtype=np.float64)
+    lse = np.empty((B, Hq, nr), dtype=np.float64)
+    rc = _load().oracle_attn_fwd_fp8(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(qs), _ptr(ks), _ptr(vs),
+                                     B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+                                     int(window), rp, nr, _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attn_fwd_fp8 rejected its arguments")
     return torch.from_numpy(o), torch.from_numpy(lse)

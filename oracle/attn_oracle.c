@@ -408,6 +408,88 @@ int oracle_decode_fp8(const uint16_t *q, const uint8_t *kcache, const uint8_t *v
     return err ? -1 : 0;
 }
 
+/*
+ * Prefill over FP8 (E4M3) Q, K and V.  The pages list FP8 among the data types of
+ * FlashAttention-3 (toolsku.com, the FlashAttention generations table) without a scale
+ * convention; this library's reading is the one of the FP8 KV cache above, extended to Q:
+ *   q[b, h, i, :] = q_scale[h] * e4m3(q8[b, h, i, :])        (one scale per query head)
+ *   k[b, g, j, :] = k_scale[g] * e4m3(k8[b, g, j, :])        (one per K/V head)
+ *   v[b, g, j, :] = v_scale[g] * e4m3(v8[b, g, j, :])
+ * and the result is the attention of these dequantized tensors: the same two passes as
+ * attend_row, written out over the dequantized values, with the causal and sliding-window
+ * rules of oracle_attn_fwd_window.  Layouts as there, with bytes in place of bf16 bits.
+ */
+static void attend_row_fp8(const uint8_t *qrow, double qs, const uint8_t *khead, double ks,
+                           const uint8_t *vhead, double vs, long nkeys, long d, double scale,
+                           const double *lut, double *qbuf, double *s, double *orow, double *lse)
+{
+    for (long t = 0; t < d; ++t) qbuf[t] = qs * lut[qrow[t]];
+    for (long t = 0; t < d; ++t) orow[t] = 0.0;
+    if (nkeys <= 0) { *lse = -INFINITY; return; }
+    for (long j = 0; j < nkeys; ++j) {
+        const uint8_t *kr = khead + j * d;
+        double acc = 0.0;
+        for (long t = 0; t < d; ++t) acc += qbuf[t] * (ks * lut[kr[t]]);
+        s[j] = scale * acc;
+    }
+    double m = s[0];
+    for (long j = 1; j < nkeys; ++j) if (s[j] > m) m = s[j];
+    double l = 0.0;
+    for (long j = 0; j < nkeys; ++j) l += exp(s[j] - m);
+    for (long j = 0; j < nkeys; ++j) {
+        double p = exp(s[j] - m) / l;
+        const uint8_t *vr = vhead + j * d;
+        for (long t = 0; t < d; ++t) orow[t] += p * (vs * lut[vr[t]]);
+    }
+    *lse = m + log(l);
+}
+
+int oracle_attn_fwd_fp8(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                        const float *q_scale, const float *k_scale, const float *v_scale,
+                        int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale, int causal,
+                        int window, const int32_t *rows, int nrows, double *o, double *lse)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    if (window < 0 || (window > 0 && !causal)) return -1;
+    double lut[256];
+    for (int x = 0; x < 256; ++x) lut[x] = oracle_e4m3_to_double((uint8_t)x);
+    const long R = Hq / Hkv;
+    const long nr = rows ? nrows : Nq;
+    const long total = (long)B * Hq * nr;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *qbuf = (double *)malloc(sizeof(double) * (size_t)d);
+        double *s = (double *)malloc(sizeof(double) * (size_t)Nk);
+        if (!qbuf || !s) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long idx = 0; idx < total; ++idx) {
+                long r = idx % nr;
+                long bh = idx / nr;
+                long h = bh % Hq;
+                long b = bh / Hq;
+                long g = h / R;
+                long i = rows ? rows[r] : r;
+                if (i < 0 || i >= Nq) { continue; }
+                const uint8_t *qrow = q + (((long)b * Hq + h) * Nq + i) * d;
+                const uint8_t *kh = k + ((long)b * Hkv + g) * (long)Nk * d;
+                const uint8_t *vh = v + ((long)b * Hkv + g) * (long)Nk * d;
+                long j0 = first_key(i, Nq, Nk, window);
+                long j1 = visible_keys(i, Nq, Nk, causal);
+                attend_row_fp8(qrow, q_scale[h], kh + j0 * d, k_scale[g], vh + j0 * d, v_scale[g],
+                               j1 > j0 ? j1 - j0 : 0, d, scale, lut, qbuf, s, o + idx * d, lse + idx);
+            }
+        }
+        free(qbuf);
+        free(s);
+    }
+    return err ? -1 : 0;
+}
+
 /* Number of OpenMP threads a parallel region would use (for reporting). */
 int oracle_num_threads(void)
 {

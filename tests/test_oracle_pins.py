@@ -416,6 +416,42 @@ def pin_fp8_decode_library_sdpa():
         assert torch.allclose(lse[b], rl[0, :, 0], atol=1e-12, rtol=0)
 
 
+def _fp8_prefill_cases():
+    # (B, Hq, Hkv, Nq, Nk, d, causal, window): MHA, GQA, chunked causal, a window
+    return [(1, 2, 2, 40, 40, 32, True, 0), (2, 4, 2, 33, 50, 16, True, 0),
+            (1, 4, 1, 20, 20, 64, False, 0), (1, 2, 1, 30, 45, 32, True, 7)]
+
+
+def pin_fp8_prefill_equals_bf16_prefill_with_power_of_two_scales():
+    """With power-of-two scales every dequantized Q, K and V value is exactly a bf16, so the
+    FP8 prefill must equal the bf16 prefill of the dequantized tensors bit for bit."""
+    for n, (B, Hq, Hkv, Nq, Nk, d, causal, W) in enumerate(_fp8_prefill_cases()):
+        w = inputs.make_fp8_prefill(B, Hq, Hkv, Nq, Nk, d, seed=82 + n, causal=causal, window=W)
+        qs = torch.tensor([2.0 ** (e % 5 - 2) for e in range(Hq)], dtype=torch.float32)
+        ks = torch.tensor([2.0 ** (1 - e % 3) for e in range(Hkv)], dtype=torch.float32)
+        vs = torch.tensor([2.0 ** (e % 4 - 3) for e in range(Hkv)], dtype=torch.float32)
+        qb, kb, vb = (_dequant(t, sc).to(torch.bfloat16) for t, sc in ((w.q, qs), (w.k, ks), (w.v, vs)))
+        assert torch.equal(qb.double(), _dequant(w.q, qs))
+        rows = torch.tensor([0, Nq // 2, Nq - 1], dtype=torch.int32)
+        for r in (None, rows):
+            o, lse = oracle.attn_fwd_fp8(w.q, w.k, w.v, qs, ks, vs, w.scale, causal, rows=r, window=W)
+            ob, lb = oracle.attn_fwd(qb, kb, vb, w.scale, causal, rows=r, window=W)
+            assert torch.equal(o, ob) and torch.equal(lse, lb)
+
+
+def pin_fp8_prefill_library_sdpa():
+    """Arbitrary per-head scales (distinct for every Q, K and V head): torch fp64 SDPA, with
+    torch's own E4M3 decoding, on the dequantized tensors."""
+    for n, (B, Hq, Hkv, Nq, Nk, d, causal, W) in enumerate(_fp8_prefill_cases()):
+        w = inputs.make_fp8_prefill(B, Hq, Hkv, Nq, Nk, d, seed=86 + n, causal=causal, window=W)
+        assert len(set(w.q_scale.tolist())) == Hq and len(set(w.k_scale.tolist() + w.v_scale.tolist())) == 2 * Hkv
+        o, lse = oracle.attn_fwd_fp8(w.q, w.k, w.v, w.q_scale, w.k_scale, w.v_scale, w.scale, causal, window=W)
+        ro, rl = _sdpa_ref(_dequant(w.q, w.q_scale), _dequant(w.k, w.k_scale), _dequant(w.v, w.v_scale),
+                           w.scale, causal, window=W)
+        assert torch.allclose(o, ro, atol=1e-12, rtol=0)
+        assert torch.allclose(lse, rl, atol=1e-12, rtol=0)
+
+
 def pin_context_parallel_merge_equals_unsplit():
     """The cache cut into R contiguous shards (some empty for short sequences), each decoded
     on its own by the C oracle and merged by merge_lse, equals the unsplit decode."""
@@ -471,6 +507,11 @@ MUTANTS = [
     ("fp8 scales swapped", "kd[e] = (double)k_scale[g] * oracle_e4m3_to_double(kh[e]);",
      "kd[e] = (double)v_scale[g] * oracle_e4m3_to_double(kh[e]);"),
     ("fp8 normaliser dropped", "double w = exp(s[j] - mx) / sum;", "double w = exp(s[j] - mx);"),
+    ("fp8 prefill q scale of the kv head", "attend_row_fp8(qrow, q_scale[h],", "attend_row_fp8(qrow, q_scale[g],"),
+    ("fp8 prefill v scale dropped", "orow[t] += p * (vs * lut[vr[t]]);", "orow[t] += p * lut[vr[t]];"),
+    ("fp8 prefill k scale from v", "acc += qbuf[t] * (ks * lut[kr[t]]);", "acc += qbuf[t] * (vs * lut[kr[t]]);"),
+    ("fp8 prefill window dropped", "long j0 = first_key(i, Nq, Nk, window);\n                long j1 = visible_keys(i, Nq, Nk, causal);\n                attend_row_fp8",
+     "long j0 = 0;\n                long j1 = visible_keys(i, Nq, Nk, causal);\n                attend_row_fp8"),
 ]
 
 
