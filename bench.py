@@ -11,7 +11,8 @@ workloads' inputs exceed the 126 MB L2, so no flush is needed between steps.
 The same line carries a ``configs`` block: every other named workload (the grouped-query
 causal prefills at 8K and 32K, the same 8K problem on (batch, sequence, heads, dim) tensors,
 sliding window, chunked prefill, paged and FP8 decode, and the small fp32-output problem)
-timed the same way, one kernel call per timed iteration, with its roofline fraction.
+timed the same way, one kernel call per timed iteration, with its roofline fraction; also
+the same two prefill problems over FP8 (E4M3) inputs.
 
 ``--gpus N``: one process per GPU.  Under torchrun the world size must equal N; started
 without torchrun, the script re-launches itself under ``torch.distributed.run`` with N local
@@ -474,7 +475,8 @@ def run_configs(dev, peaks, world):
     """Kernel times for every other named workload, one library call per timed iteration:
     prefill 1 (small, fp32 output: launch-bound), the grouped-query causal prefills 3 (also
     on (batch, sequence, heads, dim) tensors through fa_fwd_bshd) and 4, sliding window (6, 8),
-    chunked prefill (7, 8), paged decode (9) and FP8 decode (10).  Every input but prefill 1's
+    chunked prefill (7, 8), paged decode (9), FP8 decode (10) and FP8 prefill (11, 12).  Every
+    input but prefill 1's
     exceeds the 126 MB L2, so back-to-back calls do not hit in L2.  Times are the max over
     ranks; throughputs are per GPU."""
     from exact_io_aware_81_b200 import ops
@@ -516,6 +518,25 @@ def run_configs(dev, peaks, world):
             launches += 200
         res[f"workload{kid}" + ("_bshd" if bshd else "")] = entry
         del q, k, v, o, lse, w
+        torch.cuda.empty_cache()
+    # FP8 prefill (11: workload 2 in E4M3, 12: workload 3 in E4M3).  Its S = Q K^T runs at the
+    # FP8 rate and P V at the 16-bit rate, so the bf16 peak is the conservative denominator.
+    for kid in (11, 12):
+        w = inputs.workload(kid)
+        t = [x.to(dev) for x in (w.q, w.k, w.v, w.q_scale, w.k_scale, w.v_scale)]
+        B, Hq, Hkv, Nq, Nk, d = w.shape
+        o = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+        n = 10
+        ms = _time_calls(lambda: ops.fwd_fp8(*t, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream),
+                         n, stream)
+        launches += n
+        ms = max_over_ranks(ms, world, dev)
+        tf = w.flops() / (ms * 1e-3) / 1e12
+        res[f"workload{kid}"] = {"workload": w.name, "ms": ms, "tflops": tf, "frac": tf / tensor_peak,
+                                 "bound": "tensor", "algorithmic_flops": w.flops(), "kernel": PREFILL_KERNEL + " (FP8)",
+                                 "peak_note": "bf16 peak: only Q K^T runs at the FP8 rate"}
+        del t, o, lse, w
         torch.cuda.empty_cache()
     # decode over a paged cache (9) and over an FP8 cache (10): HBM-bound like decode 5
     for kid in (9, 10):

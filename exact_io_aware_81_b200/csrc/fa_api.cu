@@ -48,7 +48,7 @@ struct DeviceInfo {
     bool valid = false;
     bool sm100 = false;
     int num_sms = 0;
-    bool prefill_attr_set[2][2][2][2] = {};
+    bool prefill_attr_set[2][2][2][2][2] = {};
     bool decode_attr_set[2][4][2][2] = {};
 };
 constexpr int kMaxDevices = 64;
@@ -170,17 +170,19 @@ int encode_rows_map(CUtensorMap *m, const void *base, int D, long long rows, lon
                              dims, strides, box);
 }
 
-// A prefill operand as a 4-D (d, rows, heads, batch) bf16 tensor with boxes of `box_rows`
-// rows x 64 columns of one head, 128-byte swizzle.  The memory layout is (batch, heads,
-// rows, d), or (batch, rows, heads, d) when `bshd`: only the strides differ.
+// A prefill operand as a 4-D (d, rows, heads, batch) tensor with boxes of `box_rows` rows x
+// 128 bytes of one head (64 bf16 or 128 E4M3 columns), 128-byte swizzle.  The memory layout
+// is (batch, heads, rows, d), or (batch, rows, heads, d) when `bshd`: only the strides differ.
 int encode_heads_map(CUtensorMap *m, const void *base, int D, int rows, int heads, int batch, bool bshd,
-                     unsigned box_rows = 128)
+                     unsigned box_rows = 128, bool fp8 = false)
 {
-    const cuuint64_t row = (cuuint64_t)D * 2, plane = (cuuint64_t)rows * heads * row;
+    const cuuint64_t eb = fp8 ? 1 : 2;
+    const cuuint64_t row = (cuuint64_t)D * eb, plane = (cuuint64_t)rows * heads * row;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)batch};
     const cuuint64_t strides[3] = {bshd ? heads * row : row, bshd ? row : rows * row, plane};
-    const cuuint32_t box[4] = {64, box_rows, 1, 1};
-    return encode_map_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box);
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / eb), box_rows, 1, 1};
+    return encode_map_cached(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base,
+                             dims, strides, box);
 }
 
 // ------------------------------------------------------------------- prefill
@@ -205,14 +207,15 @@ int validate_fwd(const void *q, const void *k, const void *v, const void *o, con
     return FA_OK;
 }
 
-template <int D, bool F32, bool SPLIT, bool WINDOW>
+template <int D, bool F32, bool SPLIT, bool WINDOW, bool FP8 = false>
 int launch_prefill(const fa::PrefillParams &p, DeviceInfo *info, cudaStream_t st)
 {
-    using C = fa::prefill::Cfg<D>;
-    auto kern = fa::fa_prefill_kernel<D, F32, SPLIT, WINDOW>;
+    using C = fa::prefill::Cfg<D, FP8>;
+    static_assert(C::kSmemBytes <= 227 * 1024, "prefill shared memory");
+    auto kern = fa::fa_prefill_kernel<D, F32, SPLIT, WINDOW, FP8>;
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
-        bool &set = info->prefill_attr_set[D == 128][F32][SPLIT][WINDOW];
+        bool &set = info->prefill_attr_set[D == 128][F32][SPLIT][WINDOW][FP8];
         if (!set) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  C::kSmemBytes);
@@ -228,35 +231,52 @@ int launch_prefill(const fa::PrefillParams &p, DeviceInfo *info, cudaStream_t st
     return FA_OK;
 }
 
-// Kernel variant for one head dim and output type: P handed over in halves for head-pair
-// tiling, and the sliding-window variant only when a window is set.
-template <int D, bool F32>
+// Kernel variant for one head dim, output type and input type: P handed over in halves for
+// head-pair tiling, and the sliding-window variant only when a window is set.
+template <int D, bool F32, bool FP8 = false>
 int launch_prefill_variant(const fa::PrefillParams &p, DeviceInfo *info, cudaStream_t st)
 {
     const bool win = p.window > 0;
     if (p.head_pair)
-        return win ? launch_prefill<D, F32, true, true>(p, info, st) : launch_prefill<D, F32, true, false>(p, info, st);
-    return win ? launch_prefill<D, F32, false, true>(p, info, st) : launch_prefill<D, F32, false, false>(p, info, st);
+        return win ? launch_prefill<D, F32, true, true, FP8>(p, info, st)
+                   : launch_prefill<D, F32, true, false, FP8>(p, info, st);
+    return win ? launch_prefill<D, F32, false, true, FP8>(p, info, st)
+               : launch_prefill<D, F32, false, false, FP8>(p, info, st);
 }
+
+// FP8 inputs: E4M3 Q, K, V with per-head scales (q_scale, k_scale, v_scale non-null).
+struct Fp8Scales {
+    const float *q, *k, *v;
+};
 
 int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
              int Hkv, int Nq, int Nk, int d, float scale, int causal, int window, int o_dtype,
-             bool bshd, void *stream, int selftest_timeout)
+             bool bshd, void *stream, int selftest_timeout, const Fp8Scales *fp8 = nullptr)
 {
     int rc = validate_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, o_dtype);
     if (rc != FA_OK) return rc;
     if (window < 0) return fail(FA_ERR_INVALID, "window must be >= 0 (got %d)", window);
     if (window > 0 && !causal) return fail(FA_ERR_INVALID, "a sliding window needs causal attention");
+    if (fp8 && (!fp8->q || !fp8->k || !fp8->v)) return fail(FA_ERR_INVALID, "null scale pointer");
+    if (fp8 && d != 128) return fail(FA_ERR_UNSUPPORTED, "FP8 prefill needs d = 128 (got %d)", d);
     int dev;
     DeviceInfo *info;
     if ((rc = current_device(&dev, &info)) != FA_OK) return rc;
 
     fa::PrefillParams p;
     memset(&p, 0, sizeof p);
-    if ((rc = encode_heads_map(&p.tm_q, q, d, Nq, Hq, B, bshd)) != FA_OK) return rc;
-    if ((rc = encode_heads_map(&p.tm_k, k, d, Nk, Hkv, B, bshd)) != FA_OK) return rc;
-    if ((rc = encode_heads_map(&p.tm_v, v, d, Nk, Hkv, B, bshd)) != FA_OK) return rc;
-    if (o_dtype == FA_BF16 && (rc = encode_heads_map(&p.tm_o, o, d, Nq, Hq, B, bshd, 32)) != FA_OK) return rc;
+    const bool f8 = fp8 != nullptr;
+    if ((rc = encode_heads_map(&p.tm_q, q, d, Nq, Hq, B, bshd, 128, f8)) != FA_OK) return rc;
+    if ((rc = encode_heads_map(&p.tm_k, k, d, Nk, Hkv, B, bshd, 128, f8)) != FA_OK) return rc;
+    if ((rc = encode_heads_map(&p.tm_v, v, d, Nk, Hkv, B, bshd, 128, f8)) != FA_OK) return rc;
+    // bf16 O leaves through TMA stores, except from the FP8 kernel, which stores it directly
+    if (o_dtype == FA_BF16 && !f8 && (rc = encode_heads_map(&p.tm_o, o, d, Nq, Hq, B, bshd, 32)) != FA_OK)
+        return rc;
+    if (f8) {
+        p.q_scale = fp8->q;
+        p.k_scale = fp8->k;
+        p.v_scale = fp8->v;
+    }
     p.o = o;
     p.o_sb = (long long)Hq * Nq * d;
     p.o_sh = bshd ? d : (long long)Nq * d;
@@ -290,7 +310,10 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool f32 = o_dtype == FA_F32;
-    if (d == 128)
+    if (f8)
+        rc = f32 ? launch_prefill_variant<128, true, true>(p, info, st)
+                 : launch_prefill_variant<128, false, true>(p, info, st);
+    else if (d == 128)
         rc = f32 ? launch_prefill_variant<128, true>(p, info, st) : launch_prefill_variant<128, false>(p, info, st);
     else
         rc = f32 ? launch_prefill_variant<64, true>(p, info, st) : launch_prefill_variant<64, false>(p, info, st);
@@ -511,6 +534,15 @@ int fa_fwd_bshd(const void *q, const void *k, const void *v, void *o, float *lse
                 void *stream)
 {
     return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, o_dtype, true, stream, 0);
+}
+
+int fa_fwd_fp8(const void *q, const void *k, const void *v, const float *q_scale, const float *k_scale,
+               const float *v_scale, void *o, float *lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+               float scale, int causal, int window, int o_dtype, void *stream)
+{
+    if (window > 0 && !causal) return fail(FA_ERR_INVALID, "a sliding window needs causal attention");
+    const Fp8Scales sc{q_scale, k_scale, v_scale};
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, o_dtype, false, stream, 0, &sc);
 }
 
 int fa_fwd_selftest_timeout(const void *q, const void *k, const void *v, void *o, float *lse,

@@ -28,6 +28,12 @@
 //               sum; at the end of a unit O_s / l and LSE are written out.
 //   warps 10-11 idle (they complete the third warpgroup, which lends registers to the
 //               softmax warpgroups through setmaxnreg).
+// FP8 variant (Q, K, V in E4M3 with one scale per head; toolsku.com, FlashAttention
+// generations table, FP8 among FA3's data types): S = Q K^T runs as a kind::f8f6f4 MMA on
+// the E4M3 tiles, the head scales folded into the softmax scale; warps 10-11 widen each V
+// tile to fp16 in shared memory (bit moves, exact: fp16 = E4M3 * 2^-8), so P V stays a
+// kind::f16 MMA with P rounded to fp16 (the lazy threshold is 8, so P <= 2^8 fits fp16);
+// the epilogue applies v_scale * 2^8 / l and stores O from registers.
 // The two Q tiles of a work unit share their key/value head: two query heads of one
 // group (R even) or two consecutive row tiles of one head (otherwise).  Their MMAs are
 // interleaved S0_j, PV1_{j-1}, S1_j, PV0_j -- continued across units -- so that the
@@ -37,6 +43,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "fa_common.cuh"
 #include "ptx_sm100.cuh"
@@ -64,6 +71,7 @@ struct PrefillParams {
     float scale_log2;  // scale * log2(e)
     unsigned long long wait_limit_ns;
     int selftest_no_s_signal;  // timeout self-test: never signal a ready score tile
+    const float *q_scale, *k_scale, *v_scale;  // FP8 variant: per-head dequantization scales
 };
 
 namespace prefill {
@@ -79,20 +87,26 @@ constexpr int kRegsHigh = 216;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch budget");
 constexpr int kChunkBytes = 128 * 128;  // one 64-column (128-byte) slab of a 128-row tile
 constexpr float kLazyThreshold = 16.0f;  // log2 units: rescale only past a factor of 2^16
+constexpr float kLazyThresholdF16 = 8.0f;  // FP8 variant: P <= 2^8 must fit fp16
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int D>
+template <int D, bool FP8 = false>
 struct Cfg {
-    static constexpr int kTileBytes = 128 * D * 2;
+    static constexpr int kTileBytes = 128 * D * 2;             // a 16-bit 128-row tile
+    static constexpr int kInTileBytes = FP8 ? 128 * D : kTileBytes;  // a Q, K or V tile as loaded
     // Q is double-buffered (two sets of the unit's two Q tiles) so the next unit's Q is
-    // loaded while the current one runs; the K/V ring gets what is left of 227 KB.
-    static constexpr int kStages = (D == 128) ? 3 : 8;
+    // loaded while the current one runs; the K/V ring gets what is left of 227 KB.  FP8: K
+    // and V alternate in an even ring (K in even stages, V in odd ones) and two fp16 tiles
+    // hold the widened V.
+    static constexpr int kStages = FP8 ? 4 : (D == 128) ? 3 : 8;
     static constexpr int kQOff = 0;
-    static constexpr int kKVOff = 4 * kTileBytes;
-    static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+    static constexpr int kKVOff = 4 * kInTileBytes;
+    static constexpr int kV16Off = kKVOff + kStages * kInTileBytes;
+    static constexpr int kBarOff = kV16Off + (FP8 ? 2 * kTileBytes : 0);
     // barriers: kv_full[S], kv_empty[S], q_full[2 sets][2], q_empty[2 sets][2], s_full[2],
-    //           p_ready[2], o_done[2], o_free[2], teardown, p_half[2]
-    static constexpr int kNumBars = 2 * kStages + 19;
+    //           p_ready[2], o_done[2], o_free[2], teardown, p_half[2]; FP8: v16_full[2],
+    //           v16_empty[2]
+    static constexpr int kNumBars = 2 * kStages + 19 + (FP8 ? 4 : 0);
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 };
@@ -196,15 +210,27 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_saddr, uint
     }
 }
 
+// FP8: S = Q K^T from E4M3 tiles, one 128-byte slab each (d = 128): 4 MMAs of K = 32.
+__device__ __forceinline__ void issue_qk_fp8(uint32_t d_tmem, uint32_t q_saddr, uint32_t k_saddr)
+{
+    constexpr uint32_t idesc = ptx::idesc_f32acc(BM, BN, 0, 0, 0);  // E4M3 x E4M3
+    const uint64_t a0 = ptx::smem_desc_sw128(q_saddr, 16, 1024);
+    const uint64_t b0 = ptx::smem_desc_sw128(k_saddr, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        ptx::mma_ss_f8(d_tmem, a0 + (uint64_t)(k * 2), b0 + (uint64_t)(k * 2), idesc, k > 0 ? 1u : 0u);
+}
+
 // O (+)= P V for K steps [k_begin, k_end) of the 8 (16 keys each).  P (128 x 128 bf16)
 // is read from tensor memory, 8 columns per K step.  V is an MN-major (d contiguous) 128-byte-swizzled tile: 8-key
 // groups 1024 bytes apart (stride offset), 64-column slabs of d 16 KB apart (leading
 // offset), and a K step of 16 keys advances 2048 bytes.
-template <int D, int K_BEGIN, int K_END>
+// F16: P and V in fp16 (FP8 variant) instead of bf16.
+template <int D, int K_BEGIN, int K_END, bool F16 = false>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_saddr,
                                          bool accumulate)
 {
-    constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, D, 1);
+    constexpr uint32_t idesc = F16 ? ptx::idesc_f32acc(BM, D, 0, 0, 1) : ptx::idesc_bf16_f32(BM, D, 1);
     const uint64_t b0 = ptx::smem_desc_sw128(v_saddr, kChunkBytes, 1024);
 #pragma unroll
     for (int k = K_BEGIN; k < K_END; ++k)
@@ -222,7 +248,7 @@ constexpr int kPolyPeriod = 3;
 // p are packed as bf16 pairs into x[OUT .. OUT+NC/2) (OUT <= IN, so every score is read
 // before its slot is overwritten) and their fp32 sum is returned.  Lane pairs use packed
 // fp32x2 math.
-template <int NC, int IN, int OUT>
+template <int NC, int IN, int OUT, bool F16 = false>
 __device__ __forceinline__ float exp2_pack(uint32_t (&x)[128], float sl2, float m)
 {
     static_assert(OUT <= IN && NC % 8 == 0, "in-place packing order");
@@ -242,7 +268,7 @@ __device__ __forceinline__ float exp2_pack(uint32_t (&x)[128], float sl2, float 
             e.y = ptx::ex2(y.y);
         }
         acc[c & 3] = __fadd2_rn(acc[c & 3], e);
-        x[OUT + c] = ptx::pack_bf16x2(e.x, e.y);
+        x[OUT + c] = F16 ? ptx::pack_f16x2(e.x, e.y) : ptx::pack_bf16x2(e.x, e.y);
     }
     const float2 s01 = __fadd2_rn(acc[0], acc[1]);
     const float2 s23 = __fadd2_rn(acc[2], acc[3]);
@@ -288,6 +314,49 @@ __device__ __forceinline__ void mask_cols_below(uint32_t (&x)[128], int kbase, i
     }
 }
 
+// Four E4M3 bytes b0..b3 -> fp16 pairs (b0, b1) and (b2, b3), each value times 2^-8,
+// exactly: the bytes are reordered to b0 b2 b1 b3, then for each byte the sign moves to bit
+// 15 and exponent + mantissa to bits 7-13 of its half (the exponent biases, 7 and 15,
+// differ by 8; subnormals map to subnormals).
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t x, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t y = __byte_perm(x, 0u, 0x3120);
+    lo = ((y << 8) & 0x80008000u) | ((y << 7) & 0x3F803F80u);
+    hi = (y & 0x80008000u) | ((y >> 1) & 0x3F803F80u);
+}
+
+// Widen 64 rows (rows 64 cw .. 64 cw + 63) of a 128 x 128 E4M3 V tile (TMA-written, rows of
+// 128 bytes, 128-byte swizzle) into the fp16 tile that P V reads: two 64-column slabs, rows
+// of 128 bytes, 128-byte swizzle -- the layout of a bf16 V tile.  Lane j of a quarter-warp
+// reads chunk j of one row; lanes with chunks 4-7 write their two halves in the other order,
+// so every store of a quarter-warp hits eight different bank groups.
+__device__ __forceinline__ void widen_v_tile(const uint8_t *src, uint8_t *dst, int cw, int lane)
+{
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+        const int idx = i * 32 + lane;
+        const int r = 64 * cw + (idx >> 3);
+        const int c = idx & 7;  // dims 16c .. 16c + 15
+        const uint4 x = *reinterpret_cast<const uint4 *>(src + r * 128 + ((c ^ (r & 7)) << 4));
+        uint4 a, b;  // dims 16c .. +7 and 16c + 8 .. +15 as fp16
+        e4m3x4_to_f16(x.x, a.x, a.y);
+        e4m3x4_to_f16(x.y, a.z, a.w);
+        e4m3x4_to_f16(x.z, b.x, b.y);
+        e4m3x4_to_f16(x.w, b.z, b.w);
+        uint8_t *row = dst + (c >> 2) * kChunkBytes + r * 128;
+        const int k0 = 2 * (c & 3);
+        uint4 *pa = reinterpret_cast<uint4 *>(row + ((k0 ^ (r & 7)) << 4));
+        uint4 *pb = reinterpret_cast<uint4 *>(row + (((k0 + 1) ^ (r & 7)) << 4));
+        if (c < 4) {
+            *pa = a;
+            *pb = b;
+        } else {
+            *pb = b;
+            *pa = a;
+        }
+    }
+}
+
 // A wait that ignores the stop flag, used only to let copies and MMAs already in
 // flight finish before the CTA leaves.
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
@@ -305,13 +374,16 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, uint6
 }  // namespace prefill
 
 // SPLIT_P: hand P to the MMA warp in two halves (used for head-pair units; measured to
-// help the grouped-query tiling and to cost a little on the row-pair tiling).
-template <int D, bool OUT_F32, bool SPLIT_P, bool WINDOW>
+// help the grouped-query tiling and to cost a little on the row-pair tiling).  FP8: Q, K
+// and V in E4M3 (d = 128 only).
+template <int D, bool OUT_F32, bool SPLIT_P, bool WINDOW, bool FP8 = false>
 __global__ void __launch_bounds__(prefill::kThreads, 1)
     fa_prefill_kernel(const __grid_constant__ PrefillParams p)
 {
     using namespace prefill;
-    using C = Cfg<D>;
+    using C = Cfg<D, FP8>;
+    static_assert(!FP8 || D == 128, "FP8 prefill: head dim 128");
+    constexpr int kBoxes = FP8 ? 1 : D / 64;  // 128-byte column boxes per loaded tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -327,6 +399,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
     uint64_t *o_free = q_full + 14;
     uint64_t *teardown = q_full + 16;
     uint64_t *p_half = q_full + 17;     // [2]: first 64 keys of P_s written
+    uint64_t *v16_full = q_full + 19;   // FP8 [2]: widened V tile written (one arrive per widening warp)
+    uint64_t *v16_empty = q_full + 21;  // FP8 [2]: widened V tile read by its last P V
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
     int *stop_flag = reinterpret_cast<int *>(smem + C::kMiscOff + 4);
 
@@ -336,7 +410,14 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kStages; ++i) {
             ptx::mbar_init(&kv_full[i], 1);
-            ptx::mbar_init(&kv_empty[i], 1);
+            // FP8: the V stages (odd) are released by the two widening warps
+            ptx::mbar_init(&kv_empty[i], (FP8 && (i & 1)) ? 2 : 1);
+        }
+        if (FP8) {
+            for (int i = 0; i < 2; ++i) {
+                ptx::mbar_init(&v16_full[i], 2);
+                ptx::mbar_init(&v16_empty[i], 1);
+            }
         }
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&q_full[s], 1);
@@ -373,6 +454,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
 
     const uint32_t q_saddr0 = ptx::smem_addr(smem + C::kQOff);
     const uint32_t kv_saddr0 = ptx::smem_addr(smem + C::kKVOff);
+    const uint32_t v16_saddr0 = ptx::smem_addr(smem + C::kV16Off);
 
     if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
@@ -391,12 +473,12 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             const int qi = 2 * (int)(i & 1u) + s;
             ++q_fills[qi];
             if (leader) {
-                ptx::mbar_arrive_expect_tx(&q_full[qi], C::kTileBytes);
+                ptx::mbar_arrive_expect_tx(&q_full[qi], C::kInTileBytes);
                 const int h = s ? uw.h1 : uw.h0;
                 const int r = s ? uw.r1 : uw.r0;
-                uint8_t *dst = smem + C::kQOff + qi * C::kTileBytes;
+                uint8_t *dst = smem + C::kQOff + qi * C::kInTileBytes;
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c)
+                for (int c = 0; c < kBoxes; ++c)
                     ptx::tma_load_4d(dst + c * kChunkBytes, &p.tm_q, &q_full[qi], 64 * c, r, h, uw.b);
             }
             __syncwarp();
@@ -419,11 +501,11 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     const uint32_t ph = (kv_it / C::kStages) & 1u;
                     if (!wait_warp(&kv_empty[st], ph ^ 1u, sf)) { ok = false; break; }
                     if (leader) {
-                        ptx::mbar_arrive_expect_tx(&kv_full[st], C::kTileBytes);
-                        uint8_t *dst = smem + C::kKVOff + st * C::kTileBytes;
+                        ptx::mbar_arrive_expect_tx(&kv_full[st], C::kInTileBytes);
+                        uint8_t *dst = smem + C::kKVOff + st * C::kInTileBytes;
                         const CUtensorMap *map = kv ? &p.tm_v : &p.tm_k;
 #pragma unroll
-                        for (int c = 0; c < D / 64; ++c)
+                        for (int c = 0; c < kBoxes; ++c)
                             ptx::tma_load_4d(dst + c * kChunkBytes, map, &kv_full[st], 64 * c, BN * j, w.g, w.b);
                     }
                     __syncwarp();
@@ -472,23 +554,24 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         // has written that half of P, keys 64-127 when the whole tile is done.
         auto issue_pv_halves = [&](int s, uint32_t v_stage, bool acc, bool need_free, uint32_t fpar) -> bool {
             const uint32_t d_tmem = tmem + 256 + 128 * s, p_tmem = tmem + 128 * s;
-            const uint32_t v_saddr = kv_saddr0 + v_stage * C::kTileBytes;
+            // v_stage: the K/V ring stage of V, or (FP8) the widened V tile
+            const uint32_t v_saddr = (FP8 ? v16_saddr0 : kv_saddr0) + v_stage * C::kTileBytes;
             if (SPLIT_P) {
                 if (need_free && !wait_warp(&o_free[s], fpar, sf)) return false;
                 if (!wait_warp(&p_half[s], p_ph[s], sf)) return false;
                 ptx::tc_fence_after();
-                if (leader) issue_pv<D, 0, 4>(d_tmem, p_tmem, v_saddr, acc);
+                if (leader) issue_pv<D, 0, 4, FP8>(d_tmem, p_tmem, v_saddr, acc);
                 __syncwarp();
                 if (!wait_warp(&p_ready[s], p_ph[s], sf)) return false;
                 p_ph[s] ^= 1u;
                 ptx::tc_fence_after();
-                if (leader) issue_pv<D, 4, 8>(d_tmem, p_tmem, v_saddr, true);
+                if (leader) issue_pv<D, 4, 8, FP8>(d_tmem, p_tmem, v_saddr, true);
             } else {
                 if (!wait_warp(&p_ready[s], p_ph[s], sf)) return false;
                 p_ph[s] ^= 1u;
                 if (need_free && !wait_warp(&o_free[s], fpar, sf)) return false;
                 ptx::tc_fence_after();
-                if (leader) issue_pv<D, 0, 8>(d_tmem, p_tmem, v_saddr, acc);
+                if (leader) issue_pv<D, 0, 8, FP8>(d_tmem, p_tmem, v_saddr, acc);
             }
             __syncwarp();
             return true;
@@ -496,7 +579,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         auto issue_pv1 = [&](uint32_t v_stage, bool acc, bool need_free, uint32_t fpar, bool last) -> bool {
             if (!issue_pv_halves(1, v_stage, acc, need_free, fpar)) return false;
             if (leader) {
-                ptx::mma_commit(&kv_empty[v_stage]);
+                ptx::mma_commit(FP8 ? &v16_empty[v_stage] : &kv_empty[v_stage]);
                 if (last) ptx::mma_commit(&o_done[1]);
             }
             __syncwarp();
@@ -509,7 +592,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             const uint32_t q_par = (units >> 1) & 1u;
             uint64_t *qf = q_full + 2 * qset;
             uint64_t *qe = q_empty + 2 * qset;
-            const uint32_t q_saddr = q_saddr0 + 2 * qset * C::kTileBytes;
+            const uint32_t q_saddr = q_saddr0 + 2 * qset * C::kInTileBytes;
             if (!wait_warp(&qf[0], q_par, sf) || !wait_warp(&qf[1], q_par, sf)) break;
             ptx::tc_fence_after();
             uint32_t prev_v = 0;
@@ -517,14 +600,18 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             for (int j = w.a0; j < w.n1; ++j) {
                 const uint32_t ks = kv_it % C::kStages;
                 const uint32_t kph = (kv_it / C::kStages) & 1u;
-                const uint32_t vs = (kv_it + 1) % C::kStages;
-                const uint32_t vph = ((kv_it + 1) / C::kStages) & 1u;
+                // V of this key tile: its ring stage, or (FP8) its widened tile (alternating)
+                const uint32_t vs = FP8 ? (kv_it >> 1) & 1u : (kv_it + 1) % C::kStages;
+                const uint32_t vph = FP8 ? (kv_it >> 2) & 1u : ((kv_it + 1) / C::kStages) & 1u;
+                uint64_t *v_ready = FP8 ? &v16_full[vs] : &kv_full[vs];
+                uint64_t *v_release = FP8 ? &v16_empty[vs] : &kv_empty[vs];
                 if (!wait_warp(&kv_full[ks], kph, sf)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t k_saddr = kv_saddr0 + ks * C::kTileBytes;
+                const uint32_t k_saddr = kv_saddr0 + ks * C::kInTileBytes;
                 if (j < w.n0) {
                     if (leader) {
-                        issue_qk<D>(tmem + 0, q_saddr, k_saddr);
+                        if (FP8) issue_qk_fp8(tmem + 0, q_saddr, k_saddr);
+                        else issue_qk<D>(tmem + 0, q_saddr, k_saddr);
                         if (signal_s) ptx::mma_commit(&s_full[0]);
                         if (j == w.n0 - 1) ptx::mma_commit(&qe[0]);
                     }
@@ -538,14 +625,15 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 }
                 if (leader) {
                     if (j >= w.a1) {
-                        issue_qk<D>(tmem + 128, q_saddr + C::kTileBytes, k_saddr);
+                        if (FP8) issue_qk_fp8(tmem + 128, q_saddr + C::kInTileBytes, k_saddr);
+                        else issue_qk<D>(tmem + 128, q_saddr + C::kInTileBytes, k_saddr);
                         if (signal_s) ptx::mma_commit(&s_full[1]);
                     }
                     ptx::mma_commit(&kv_empty[ks]);
                     if (j == w.n1 - 1) ptx::mma_commit(&qe[1]);
                 }
                 __syncwarp();
-                if (!wait_warp(&kv_full[vs], vph, sf)) { ok = false; break; }
+                if (!wait_warp(v_ready, vph, sf)) { ok = false; break; }
                 if (j < w.n0) {
                     if (!issue_pv_halves(0, vs, j > w.a0, j == w.a0, free_par)) { ok = false; break; }
                     if (leader && j == w.n0 - 1) ptx::mma_commit(&o_done[0]);
@@ -553,7 +641,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 }
                 // a V tile that Q tile 1 never reads is released here (sliding window)
                 if (j < w.a1) {
-                    if (leader) ptx::mma_commit(&kv_empty[vs]);
+                    if (leader) ptx::mma_commit(v_release);
                     __syncwarp();
                 }
                 prev_v = vs;
@@ -582,7 +670,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + 128u * s;        // S_s, and P_s over it
         const uint32_t tO = tmem + lane_base + 256u + 128u * s;  // O_s
-        const float sl2 = p.scale_log2;
+        float sl2 = p.scale_log2;
         uint32_t s_ph = 0, units = 0;
         Unit w;
         for (int u = next_unit<WINDOW>(p, 2 * (int)blockIdx.x, w); u >= 0; u = next_unit<WINDOW>(p, unit_step(u), w)) {
@@ -593,6 +681,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             const int row = r0 + tid;
             const int lim = p.causal ? min(row + (p.Nk - p.Nq), p.Nk - 1) : p.Nk - 1;
             const int first = WINDOW ? row + (p.Nk - p.Nq) - p.window + 1 : 0;
+            // FP8: the scores are products of E4M3 codes; the head scales join the softmax scale
+            if (FP8) sl2 = p.scale_log2 * p.q_scale[h] * p.k_scale[w.g];
             // l: sum of the fp32 weights (gives the LSE).  lo: normaliser of O, the same sum
             // corrected, tile by tile, by the bf16 rounding of the tile's largest weight --
             // the rounding the P V product actually saw.  For a row dominated by one key
@@ -620,7 +710,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 mx = fmaxf(row_max64<0>(x), row_max64<64>(x)) * sl2;
                 if (j == a) {
                     m = mx;  // O is not written yet: the first P V overwrites it
-                } else if (mx - m > kLazyThreshold) {
+                } else if (mx - m > (FP8 ? kLazyThresholdF16 : kLazyThreshold)) {
                     // (also taken when m is still -inf: the row's window had not started)
                     alpha = ptx::ex2(m - mx);
                     m = mx;
@@ -651,22 +741,23 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     // the first 64 keys of P are handed to the MMA warp while the second
                     // half is still being computed
                     rescale_o();
-                    sum = exp2_pack<64, 0, 0>(x, sl2, mref);
+                    sum = exp2_pack<64, 0, 0, FP8>(x, sl2, mref);
                     ptx::tmem_st32(tS + 0, &x[0]);
                     ptx::tmem_wait_st();
                     ptx::tc_fence_before();
                     ptx::mbar_arrive(&p_half[s]);
-                    sum += exp2_pack<64, 64, 32>(x, sl2, mref);
+                    sum += exp2_pack<64, 64, 32, FP8>(x, sl2, mref);
                     ptx::tmem_st32(tS + 32, &x[32]);
                 } else {
-                    sum = exp2_pack<64, 0, 0>(x, sl2, mref) + exp2_pack<64, 64, 32>(x, sl2, mref);
+                    sum = exp2_pack<64, 0, 0, FP8>(x, sl2, mref) + exp2_pack<64, 64, 32, FP8>(x, sl2, mref);
                     ptx::tmem_st32(tS + 0, &x[0]);
                     ptx::tmem_st32(tS + 32, &x[32]);
                     rescale_o();
                 }
                 ptx::tmem_wait_st();
                 const float p_top = ptx::ex2(mx - mref);  // the tile's largest weight (0 if masked)
-                const float p_top_bf = __uint_as_float(ptx::pack_bf16x2(p_top, 0.f) << 16);
+                const float p_top_bf = FP8 ? __half2float(__float2half_rn(p_top))
+                                           : __uint_as_float(ptx::pack_bf16x2(p_top, 0.f) << 16);
                 l = l * alpha + sum;
                 lo = lo * alpha + sum + (p_top_bf - p_top);
                 ptx::tc_fence_before();
@@ -682,7 +773,8 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             if (!wait_warp(&o_done[s], units & 1u, sf)) break;
             ptx::tc_fence_after();
             const bool valid = row < p.Nq;
-            const float inv_l = 1.f / lo;
+            // FP8: the widened V holds E4M3 codes times 2^-8; v_scale and 2^8 restore V
+            const float inv_l = FP8 ? p.v_scale[w.g] * 256.f / lo : 1.f / lo;
             const size_t orow = ((size_t)w.b * p.Hq + h) * (size_t)p.Nq + (size_t)(valid ? row : 0);  // LSE index
             const int qi = 2 * (int)(units & 1u) + s;
             uint32_t ov[D];
@@ -701,6 +793,22 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                                              __uint_as_float(ov[4 * e + 1]) * inv_l,
                                              __uint_as_float(ov[4 * e + 2]) * inv_l,
                                              __uint_as_float(ov[4 * e + 3]) * inv_l);
+                }
+                if (lane == 0) ptx::mbar_arrive(&q_empty[qi]);
+            } else if (FP8) {
+                // bf16 O stored from registers (an E4M3 Q slot is too small to stage it)
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + w.b * p.o_sb +
+                                                           h * p.o_sh + (long long)row * p.o_sn);
+#pragma unroll
+                    for (int e = 0; e < D / 8; ++e) {
+                        uint4 v4;
+                        v4.x = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
+                        v4.y = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
+                        v4.z = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
+                        v4.w = ptx::pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
+                        dst[e] = v4;
+                    }
                 }
                 if (lane == 0) ptx::mbar_arrive(&q_empty[qi]);
             } else {
@@ -733,11 +841,41 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             if (valid) p.lse[orow] = (m + ptx::lg2(l)) * kLn2;
             ++units;
         }
-        if (!OUT_F32 && lane == 0) ptx::bulk_wait_group0();  // stores complete before exit
+        if (!OUT_F32 && !FP8 && lane == 0) ptx::bulk_wait_group0();  // stores complete before exit
     }
 
     else {
         ptx::regs_decrease<kRegsLow>();
+        if (FP8) {
+            // -------------------------------------------------------- V widening (FP8)
+            // Warps 10 and 11 follow the producer's key-tile order and turn each E4M3 V
+            // tile (odd ring stage) into the fp16 tile P V reads, rows 64 (warp - 10) on.
+            const int cw = warp - 10;
+            uint32_t kv_it = 0;
+            bool ok = true;
+            Unit w;
+            for (int u = next_unit<WINDOW>(p, 2 * (int)blockIdx.x, w); ok && u >= 0;
+                 u = next_unit<WINDOW>(p, unit_step(u), w)) {
+                for (int j = w.a0; j < w.n1; ++j, kv_it += 2) {
+                    const uint32_t st = (kv_it + 1) % C::kStages;
+                    const uint32_t ph = ((kv_it + 1) / C::kStages) & 1u;
+                    const uint32_t vb = (kv_it >> 1) & 1u;
+                    const uint32_t vpar = (kv_it >> 2) & 1u;
+                    if (!wait_warp(&kv_full[st], ph, sf) || !wait_warp(&v16_empty[vb], vpar ^ 1u, sf)) {
+                        ok = false;
+                        break;
+                    }
+                    widen_v_tile(smem + C::kKVOff + st * C::kInTileBytes, smem + C::kV16Off + vb * C::kTileBytes,
+                                 cw, lane);
+                    ptx::fence_proxy_async_smem();  // the tensor core reads these through the async proxy
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::mbar_arrive(&v16_full[vb]);
+                        ptx::mbar_arrive(&kv_empty[st]);
+                    }
+                }
+            }
+        }
     }
     __syncwarp();
     ptx::tc_fence_before();

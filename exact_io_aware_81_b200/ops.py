@@ -36,6 +36,7 @@ SIGNATURES = {
     "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_fwd_bshd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
+    "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
     "fa_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
@@ -219,6 +220,40 @@ def fwd_window(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int,
         raise ValueError("window must be >= 1")
     return fwd(q, k, v, causal=True, scale=scale, out_dtype=out_dtype, out=out, lse=lse,
                stream=stream, window=int(window))
+
+
+def fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_scale: torch.Tensor,
+            k_scale: torch.Tensor, v_scale: torch.Tensor, causal: bool = False,
+            scale: Optional[float] = None, out_dtype: torch.dtype = torch.bfloat16,
+            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+            stream=None, window: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Attention forward over FP8 E4M3 inputs: q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d) uint8 bytes
+    with fp32 per-head scales q_scale (Hq), k_scale/v_scale (Hkv) -> (o, lse).  The value
+    of a q row of head h is q_scale[h] * e4m3(bytes); likewise K and V.  ``scale`` defaults
+    to 1/sqrt(d); d must be 128."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n, torch.uint8, 4)
+    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        _require(t, n, torch.float32, 1)
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if Bk != B or dk != d or tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    if q_scale.numel() != Hq or k_scale.numel() != Hkv or v_scale.numel() != Hkv:
+        raise ValueError("q_scale must have Hq entries, k_scale and v_scale Hkv entries")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    out, lse = _fwd_outputs(q, (B, Hq, Nq, d), (B, Hq, Nq), out_dtype, out, lse)
+    odt = FA_F32 if out_dtype == torch.float32 else FA_BF16
+    with _on_device(q, k, v, q_scale, k_scale, v_scale, out, lse) as dev:
+        rc = load().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), q_scale.data_ptr(),
+                               k_scale.data_ptr(), v_scale.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                               B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), int(window), odt,
+                               _stream_handle(stream, dev))
+    _check(rc)
+    return out, lse
 
 
 def decode_workspace_size(B: int, Hq: int, Nmax: int, d: int) -> int:

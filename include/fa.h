@@ -90,6 +90,30 @@ FA_API int fa_fwd_window(const void *q, const void *k, const void *v, void *o, f
                   int o_dtype, void *stream);
 
 /*
+ * Forward attention over FP8 (E4M3) Q, K and V.  FP8 is among the data types of
+ * FlashAttention-3 in the toolsku.com "attention mechanism evolution" FlashAttention
+ * generations table; the pages fix no scale convention, and this library's is one
+ * dequantization scale per head:
+ *   q[b,h,i,:] = q_scale[h] * e4m3(q8[b,h,i,:]),  k[b,g,j,:] = k_scale[g] * e4m3(k8[b,g,j,:]),
+ *   v[b,g,j,:] = v_scale[g] * e4m3(v8[b,g,j,:]),
+ * and the result is the attention of these tensors (masks, alignment and LSE as fa_fwd_ex
+ * and fa_fwd_window).
+ *   q  (B, Hq,  Nq, d) uint8 E4M3 bytes ("e4m3fn": bias 7, no infinities), device
+ *   k, v (B, Hkv, Nk, d) uint8 E4M3 bytes, device
+ *   q_scale (Hq), k_scale (Hkv), v_scale (Hkv): fp32, device
+ *   o   (B, Hq, Nq, d) written, bf16 or fp32 (o_dtype); lse (B, Hq, Nq) fp32 written
+ *   causal, window: as fa_fwd_window (window 0 for none; a window needs causal != 0).
+ * S = Q K^T is computed exactly in fp32 from the E4M3 codes on the tensor cores; P is
+ * rounded to fp16 for P V (V widened to fp16 on chip, exactly).  d must be 128
+ * (FA_ERR_UNSUPPORTED otherwise); a null scale pointer is FA_ERR_INVALID.  E4M3 NaN bytes
+ * are not special-cased.  Ownership, alignment and the other errors as fa_fwd_ex.
+ */
+FA_API int fa_fwd_fp8(const void *q, const void *k, const void *v, const float *q_scale,
+                      const float *k_scale, const float *v_scale, void *o, float *lse, int B, int Hq,
+                      int Hkv, int Nq, int Nk, int d, float scale, int causal, int window, int o_dtype,
+                      void *stream);
+
+/*
  * Forward attention on (batch, sequence, heads, dim) tensors, the layout of the
  * flash_attn_func call in toolsku.com "attention mechanism evolution", FlashAttention
  * usage example (its layer views the projections as (B, S, H, d) and passes them on with

@@ -252,3 +252,37 @@ def _fwd_bshd(lib, **kw):
 def test_fwd_bshd_rejects(lib, kw, status):
     assert _fwd_bshd(lib, **kw) == status
 
+
+
+def _fwd_fp8(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, qs=FAKE, ks=FAKE, vs=FAKE, o=FAKE, lse=FAKE, B=1, Hq=4, Hkv=2, Nq=8,
+             Nk=8, d=128, scale=0.125, causal=1, window=0, dt=0)
+    a.update(kw)
+    return lib.fa_fwd_fp8(a["q"], a["k"], a["v"], a["qs"], a["ks"], a["vs"], a["o"], a["lse"], a["B"], a["Hq"],
+                          a["Hkv"], a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"], a["window"], a["dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(qs=None), ops.FA_ERR_INVALID),
+    (dict(ks=None), ops.FA_ERR_INVALID),
+    (dict(vs=None), ops.FA_ERR_INVALID),
+    (dict(q=None), ops.FA_ERR_INVALID),
+    (dict(window=-2), ops.FA_ERR_INVALID),
+    (dict(causal=0, window=4), ops.FA_ERR_INVALID),    # a window needs causal attention
+    (dict(Nq=9, Nk=8), ops.FA_ERR_INVALID),            # causal needs Nq <= Nk
+    (dict(Hq=6, Hkv=4), ops.FA_ERR_INVALID),
+    (dict(dt=5), ops.FA_ERR_INVALID),
+    (dict(scale=-0.5), ops.FA_ERR_INVALID),
+    (dict(d=64), ops.FA_ERR_UNSUPPORTED),              # FP8 rows are one 128-byte box
+    (dict(v=FAKE + 4), ops.FA_ERR_UNSUPPORTED),
+])
+def test_fwd_fp8_rejects(lib, kw, status):
+    assert _fwd_fp8(lib, **kw) == status
+    assert lib.fa_last_error_message().decode() != ""
+
+
+def test_decode_selftest_timeout_rejects_one_scale(lib):
+    ws = lib.fa_decode_workspace_size(2, 8, 300, 128)
+    rc = lib.fa_decode_selftest_timeout(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, 2, 8, 2, 300, 128, 0.1,
+                                        FAKE, ws, None)
+    assert rc == ops.FA_ERR_INVALID
