@@ -269,9 +269,8 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     if ((rc = encode_heads_map(&p.tm_q, q, d, Nq, Hq, B, bshd, 128, f8)) != FA_OK) return rc;
     if ((rc = encode_heads_map(&p.tm_k, k, d, Nk, Hkv, B, bshd, 128, f8)) != FA_OK) return rc;
     if ((rc = encode_heads_map(&p.tm_v, v, d, Nk, Hkv, B, bshd, 128, f8)) != FA_OK) return rc;
-    // bf16 O leaves through TMA stores, except from the FP8 kernel, which stores it directly
-    if (o_dtype == FA_BF16 && !f8 && (rc = encode_heads_map(&p.tm_o, o, d, Nq, Hq, B, bshd, 32)) != FA_OK)
-        return rc;
+    // bf16 O leaves through TMA stores of one warp's 32 rows
+    if (o_dtype == FA_BF16 && (rc = encode_heads_map(&p.tm_o, o, d, Nq, Hq, B, bshd, 32)) != FA_OK) return rc;
     if (f8) {
         p.q_scale = fp8->q;
         p.k_scale = fp8->k;
