@@ -251,7 +251,8 @@ struct Fp8Scales {
 
 int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
              int Hkv, int Nq, int Nk, int d, float scale, int causal, int window, int o_dtype,
-             bool bshd, void *stream, int selftest_timeout, const Fp8Scales *fp8 = nullptr)
+             bool bshd, void *stream, int selftest_timeout, const Fp8Scales *fp8 = nullptr,
+             bool debug_bounds_selftest = false)
 {
     int rc = validate_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, o_dtype);
     if (rc != FA_OK) return rc;
@@ -306,6 +307,8 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     p.scale_log2 = scale * 1.4426950408889634f;
     p.wait_limit_ns = g_wait_limit_ns;
     p.selftest_no_s_signal = selftest_timeout;
+    // the debug build's bounds self-test moves every LSE index past the end of its buffer
+    p.debug_lse_offset = debug_bounds_selftest ? (long long)B * Hq * Nq : 0;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool f32 = o_dtype == FA_F32;
@@ -745,6 +748,8 @@ int fa_get_error(void *stream)
     if (word & fa::kErrSeqlenRange) return fail(FA_ERR_DEVICE_ARG, "seqlens held a value outside [0, Nmax]");
     if (word & fa::kErrPageRange)
         return fail(FA_ERR_DEVICE_ARG, "the block table held a page outside [0, num_pages)");
+    if (word & fa::kErrDebugBounds)
+        return fail(FA_ERR_DEBUG_CHECK, "a kernel's global-memory index failed its bounds check (access skipped)");
     return ok();
 }
 
@@ -760,6 +765,7 @@ const char *fa_status_str(int status)
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
     case FA_ERR_DEVICE_ARG: return "FA_ERR_DEVICE_ARG";
+    case FA_ERR_DEBUG_CHECK: return "FA_ERR_DEBUG_CHECK";
     default: return "FA_ERR_UNKNOWN";
     }
 }
@@ -767,5 +773,16 @@ const char *fa_status_str(int status)
 const char *fa_last_error_message(void) { return g_msg; }
 
 int fa_version(void) { return kVersion; }
+
+int fa_build_flags(void) { return fa::kDebugChecks ? 1 : 0; }
+
+int fa_debug_selftest_bounds(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                             int Hkv, int Nq, int Nk, int d, float scale, int causal, void *stream)
+{
+    if (!fa::kDebugChecks)
+        return fail(FA_ERR_UNSUPPORTED, "bounds checks are compiled only into the debug build (libfa_debug.so)");
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, FA_BF16, false, stream, 0, nullptr,
+                    true);
+}
 
 }  // extern "C"

@@ -12,12 +12,33 @@ enum : unsigned int {
     kErrTimeout = 1u,      // a pipeline wait exceeded its limit
     kErrSeqlenRange = 2u,  // a decode length was outside [0, Nmax] and was clamped
     kErrPageRange = 4u,    // a block-table entry was outside [0, num_pages); its keys read as 0
+    kErrDebugBounds = 8u,  // debug builds: an address computed by a kernel failed its bounds check
 };
 
 // One word per process, in the library's own device memory.
 __device__ unsigned int g_error_word = 0;
 
 __device__ __forceinline__ void raise_error(unsigned int bit) { atomicOr(&g_error_word, bit); }
+
+// Debug builds (compiled with FA_DEBUG_CHECKS): every global-memory index that a kernel
+// computes by hand (outputs, partials, scales, block-table and q rows) is checked against
+// the size of its buffer before the access; a failed check records kErrDebugBounds and the
+// access is skipped, so a bad index is reported instead of touching memory outside the
+// buffer.  (TMA copies are bounds-checked by the copy engine itself.)  In release builds the
+// check is the constant true and costs nothing.
+#ifdef FA_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
+__device__ __forceinline__ bool in_bounds(long long idx, long long n)
+{
+    if (!kDebugChecks) return true;
+    if (idx >= 0 && idx < n) return true;
+    raise_error(kErrDebugBounds);
+    return false;
+}
 
 // Per-CTA stop flag (in shared memory): set by the first role whose wait runs out, read
 // by every other role at each wait so that the whole CTA winds down together.

@@ -300,7 +300,8 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             if (PAGED) {
                 first_lp = start / p.page_size;
                 const int lp = first_lp + lane;
-                if (lp <= (start + n - 1) / p.page_size) {
+                if (lp <= (start + n - 1) / p.page_size &&
+                    in_bounds((long long)b * p.max_pages + lp, (long long)p.B * p.max_pages)) {
                     my_page = p.block_table[(size_t)b * p.max_pages + lp];
                     if (my_page < 0 || my_page >= p.num_pages) {
                         raise_error(kErrPageRange);
@@ -373,12 +374,13 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
         // that their latency overlaps the previous item's passes: r[2ks], r[2ks+1] = dims
         // 16ks + 2tig + {0,1}, 16ks + 8 + 2tig + {0,1}.
         auto load_q = [&](int qb_, int qhg, uint32_t (&r)[2 * KSTEPS]) {
-            const __nv_bfloat16 *qrow = p.q + ((size_t)qb_ * p.Hq + qhg * RG + (row_real ? gid : 0)) * D;
-            const uint32_t *qw = reinterpret_cast<const uint32_t *>(qrow);
+            const long long qr = (long long)qb_ * p.Hq + qhg * RG + (row_real ? gid : 0);
+            const bool use = row_real && in_bounds(qr, (long long)p.B * p.Hq);
+            const uint32_t *qw = reinterpret_cast<const uint32_t *>(p.q + qr * D);
 #pragma unroll
             for (int ks = 0; ks < KSTEPS; ++ks) {
-                r[2 * ks] = row_real ? qw[8 * ks + tig] : 0u;
-                r[2 * ks + 1] = row_real ? qw[8 * ks + 4 + tig] : 0u;
+                r[2 * ks] = use ? qw[8 * ks + tig] : 0u;
+                r[2 * ks + 1] = use ? qw[8 * ks + 4 + tig] : 0u;
             }
         };
         int b = 0, hg = 0, start = 0, n = 0;
@@ -515,24 +517,30 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             {
                 const float f0 = hc0 < RG ? 1.f / l_sm[hc0] : 0.f;
                 const float f1 = hc1 < RG ? 1.f / l_sm[hc1] : 0.f;
-                float *dst0 = p.part_o + (((size_t)b * p.Hq + h0 + hc0) * p.S_max + chunk) * D;
-                float *dst1 = p.part_o + (((size_t)b * p.Hq + h0 + hc1) * p.S_max + chunk) * D;
+                const long long n_parts = (long long)p.B * p.Hq * p.S_max;  // partial rows in the workspace
+                const long long r0p = ((long long)b * p.Hq + h0 + hc0) * p.S_max + chunk;
+                const long long r1p = ((long long)b * p.Hq + h0 + hc1) * p.S_max + chunk;
+                const bool w0 = hc0 < RG && in_bounds(r0p, n_parts), w1 = hc1 < RG && in_bounds(r1p, n_parts);
+                float *dst0 = p.part_o + r0p * D;
+                float *dst1 = p.part_o + r1p * D;
 #pragma unroll
                 for (int i = 0; i < VT; ++i) {
                     const int dim = 16 * (VT * warp + i) + gid;      // rows gid / gid + 8 = dims +0 / +8
-                    if (hc0 < RG) {
+                    if (w0) {
                         dst0[dim] = acc[i][0] * f0;
                         dst0[dim + 8] = acc[i][2] * f0;
                     }
-                    if (hc1 < RG) {
+                    if (w1) {
                         dst1[dim] = acc[i][1] * f1;
                         dst1[dim + 8] = acc[i][3] * f1;
                     }
                 }
             }
-            if (threadIdx.x < RG)
-                p.part_lse[((size_t)b * p.Hq + h0 + threadIdx.x) * p.S_max + chunk] =
-                    m_sm[threadIdx.x] + ptx::lg2(l_sm[threadIdx.x]);
+            if (threadIdx.x < RG) {
+                const long long rp = ((long long)b * p.Hq + h0 + threadIdx.x) * p.S_max + chunk;
+                if (in_bounds(rp, (long long)p.B * p.Hq * p.S_max))
+                    p.part_lse[rp] = m_sm[threadIdx.x] + ptx::lg2(l_sm[threadIdx.x]);
+            }
             // scores and m/l are rewritten by the next item
             if (!gb.sync(sf)) break;
             b = nb;
@@ -622,7 +630,8 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
                 first_lp[w] = start[w] / p.page_size;
                 const int lp = first_lp[w] + lane;
                 int pg = 0;
-                if (lp <= (start[w] + n[w] - 1) / p.page_size) {
+                if (lp <= (start[w] + n[w] - 1) / p.page_size &&
+                    in_bounds((long long)b * p.max_pages + lp, (long long)p.B * p.max_pages)) {
                     pg = p.block_table[(size_t)b * p.max_pages + lp];
                     if (pg < 0 || pg >= p.num_pages) {
                         raise_error(kErrPageRange);
@@ -739,15 +748,17 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
         // ahead, so that their latency overlaps the previous item: r[2ks], r[2ks+1] = dims
         // 16ks + 4tig + {0,1}, 16ks + 4tig + {2,3}.
         auto load_q = [&](int qb_, int qhg, uint32_t (&r)[2 * KSTEPS], float &ksc) {
-            const __nv_bfloat16 *qrow = p.q + ((size_t)qb_ * p.Hq + qhg * RG + (row_real ? gid : 0)) * D;
+            const long long qr = (long long)qb_ * p.Hq + qhg * RG + (row_real ? gid : 0);
+            const bool use = row_real && in_bounds(qr, (long long)p.B * p.Hq);
+            const __nv_bfloat16 *qrow = p.q + qr * D;
 #pragma unroll
             for (int ks = 0; ks < KSTEPS; ++ks) {
-                const uint2 raw = row_real ? *reinterpret_cast<const uint2 *>(qrow + 16 * ks + 4 * tig)
-                                           : make_uint2(0u, 0u);
+                const uint2 raw = use ? *reinterpret_cast<const uint2 *>(qrow + 16 * ks + 4 * tig)
+                                      : make_uint2(0u, 0u);
                 r[2 * ks] = raw.x;
                 r[2 * ks + 1] = raw.y;
             }
-            ksc = p.k_scale[qhg * RG / p.R];
+            ksc = in_bounds(qhg * RG / p.R, p.Hkv) ? p.k_scale[qhg * RG / p.R] : 0.f;
         };
         const int wid = warp * (int)gridDim.x + (int)blockIdx.x;
         int b = 0, hg = 0, start = 0, n = 0;
@@ -934,20 +945,24 @@ __global__ void __launch_bounds__(decode::kThreads, decode::kCtasPerSm)
             }
             const int chunk = start / kChunk;
             // acc[i][0..1]: heads 2tig / 2tig+1 of tile row gid; acc[i][2..3]: of row gid + 8
-            const float f0 = 256.f * p.v_scale[g] / l0;
-            const float f1 = 256.f * p.v_scale[g] / l1;
-            float *dst0 = p.part_o + (((size_t)b * p.Hq + h0 + hc0) * p.S_max + chunk) * D;
-            float *dst1 = p.part_o + (((size_t)b * p.Hq + h0 + hc1) * p.S_max + chunk) * D;
+            const float vsc = in_bounds(g, p.Hkv) ? p.v_scale[g] : 0.f;
+            const float f0 = 256.f * vsc / l0;
+            const float f1 = 256.f * vsc / l1;
+            const long long n_parts = (long long)p.B * p.Hq * p.S_max;  // partial rows in the workspace
+            const long long r0p = ((long long)b * p.Hq + h0 + hc0) * p.S_max + chunk;
+            const long long r1p = ((long long)b * p.Hq + h0 + hc1) * p.S_max + chunk;
+            const bool w0 = hc0 < RG && in_bounds(r0p, n_parts), w1 = hc1 < RG && in_bounds(r1p, n_parts);
+            float *dst0 = p.part_o + r0p * D;
+            float *dst1 = p.part_o + r1p * D;
 #pragma unroll
             for (int i = 0; i < VT; ++i) {
                 const int dim = 16 * i + 2 * gid;  // rows gid / gid + 8 = dims +0 / +1
-                if (hc0 < RG) *reinterpret_cast<float2 *>(dst0 + dim) = make_float2(acc[i][0] * f0, acc[i][2] * f0);
-                if (hc1 < RG) *reinterpret_cast<float2 *>(dst1 + dim) = make_float2(acc[i][1] * f1, acc[i][3] * f1);
+                if (w0) *reinterpret_cast<float2 *>(dst0 + dim) = make_float2(acc[i][0] * f0, acc[i][2] * f0);
+                if (w1) *reinterpret_cast<float2 *>(dst1 + dim) = make_float2(acc[i][1] * f1, acc[i][3] * f1);
             }
             if (gid == 0) {
-                const size_t base = ((size_t)b * p.Hq + h0) * p.S_max + chunk;
-                if (hc0 < RG) p.part_lse[base + (size_t)hc0 * p.S_max] = m0 + ptx::lg2(l0);
-                if (hc1 < RG) p.part_lse[base + (size_t)hc1 * p.S_max] = m1 + ptx::lg2(l1);
+                if (w0) p.part_lse[r0p] = m0 + ptx::lg2(l0);
+                if (w1) p.part_lse[r1p] = m1 + ptx::lg2(l1);
             }
             b = nb;
             hg = nhg;
@@ -982,8 +997,10 @@ __global__ void __launch_bounds__(32 * kMergeWarps) fa_decode_merge_kernel(const
     const int lane = threadIdx.x & 31;
     const size_t bh = blockIdx.x;
     const int b = (int)(bh / p.Hq);
+    if (!in_bounds((long long)bh, (long long)p.B * p.Hq)) return;  // (whole CTA: uniform)
     const int L = clamp_len(p.seqlens[b], p.Nmax);
     const int S = (L + kChunk - 1) / kChunk;
+    if (!in_bounds(S, (long long)p.S_max + 1)) return;
     const float *pl = p.part_lse + bh * p.S_max;
     const float *po = p.part_o + bh * p.S_max * D;
     if (S == 0) {

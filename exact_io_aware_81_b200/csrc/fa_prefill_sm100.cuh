@@ -72,6 +72,7 @@ struct PrefillParams {
     unsigned long long wait_limit_ns;
     int selftest_no_s_signal;  // timeout self-test: never signal a ready score tile
     const float *q_scale, *k_scale, *v_scale;  // FP8 variant: per-head dequantization scales
+    long long debug_lse_offset;  // debug builds' bounds self-test: added to every LSE index (else 0)
 };
 
 namespace prefill {
@@ -685,7 +686,10 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             const int lim = p.causal ? min(row + (p.Nk - p.Nq), p.Nk - 1) : p.Nk - 1;
             const int first = WINDOW ? row + (p.Nk - p.Nq) - p.window + 1 : 0;
             // FP8: the scores are products of E4M3 codes; the head scales join the softmax scale
-            if (FP8) sl2 = p.scale_log2 * p.q_scale[h] * p.k_scale[w.g];
+            if (FP8) {
+                const bool okq = in_bounds(h, p.Hq), okk = in_bounds(w.g, p.Hkv);
+                sl2 = p.scale_log2 * (okq ? p.q_scale[h] : 1.f) * (okk ? p.k_scale[w.g] : 1.f);
+            }
             // l: sum of the fp32 weights (gives the LSE).  lo: normaliser of O, the same sum
             // corrected, tile by tile, by the bf16 rounding of the tile's largest weight --
             // the rounding the P V product actually saw.  For a row dominated by one key
@@ -777,8 +781,9 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             ptx::tc_fence_after();
             const bool valid = row < p.Nq;
             // FP8: the widened V holds the E4M3 codes; v_scale restores V
-            const float inv_l = FP8 ? p.v_scale[w.g] / lo : 1.f / lo;
-            const size_t orow = ((size_t)w.b * p.Hq + h) * (size_t)p.Nq + (size_t)(valid ? row : 0);  // LSE index
+            const float inv_l = FP8 ? (in_bounds(w.g, p.Hkv) ? p.v_scale[w.g] : 1.f) / lo : 1.f / lo;
+            long long orow = ((long long)w.b * p.Hq + h) * (long long)p.Nq + (valid ? row : 0);  // LSE index
+            if (kDebugChecks) orow += p.debug_lse_offset;
             const int qi = 2 * (int)(units & 1u) + s;
             uint32_t ov[D];
 #pragma unroll
@@ -787,9 +792,9 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
             ptx::tc_fence_before();
             ptx::mbar_arrive(&o_free[s]);
             if (OUT_F32) {
-                if (valid) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + w.b * p.o_sb + h * p.o_sh +
-                                                             (long long)row * p.o_sn);
+                const long long ooff = w.b * p.o_sb + h * p.o_sh + (long long)row * p.o_sn;
+                if (valid && in_bounds(ooff + D - 1, (long long)p.B * p.Hq * p.Nq * D)) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + ooff);
 #pragma unroll
                     for (int e = 0; e < D / 4; ++e)
                         dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
@@ -817,7 +822,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     }
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0 && r0 + wr < p.Nq) {  // (rows past Nq are never stored)
+                    if (lane == 0 && r0 + wr < p.Nq && in_bounds(h, p.Hq) && in_bounds(w.b, p.B)) {  // (rows past Nq are never stored)
                         ptx::tma_store_4d(&p.tm_o, stage + wr * 128, 64 * c, r0 + wr, h, w.b);
                         ptx::bulk_commit_group();
                         ptx::bulk_wait_group_read0();  // the slab's rows are restaged next round
@@ -842,7 +847,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                 __syncwarp();
                 if (lane == 0) {
                     const int wr = 32 * (warp & 3);  // this warp's rows of the tile
-                    if (r0 + wr < p.Nq) {            // (rows past Nq are never stored)
+                    if (r0 + wr < p.Nq && in_bounds(h, p.Hq) && in_bounds(w.b, p.B)) {  // (rows past Nq are never stored)
 #pragma unroll
                         for (int c = 0; c < D / 64; ++c)
                             ptx::tma_store_4d(&p.tm_o, stage + c * kChunkBytes + wr * 128, 64 * c, r0 + wr, h, w.b);
@@ -852,7 +857,7 @@ __global__ void __launch_bounds__(prefill::kThreads, 1)
                     ptx::mbar_arrive(&q_empty[qi]);
                 }
             }
-            if (valid) p.lse[orow] = (m + ptx::lg2(l)) * kLn2;
+            if (valid && in_bounds(orow, (long long)p.B * p.Hq * p.Nq)) p.lse[orow] = (m + ptx::lg2(l)) * kLn2;
             ++units;
         }
         if (!OUT_F32 && lane == 0) ptx::bulk_wait_group0();  // stores complete before exit

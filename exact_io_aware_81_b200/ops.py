@@ -17,7 +17,8 @@ from typing import Optional, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfa.so")
+# FA_LIBRARY selects another build of the library, e.g. the debug build libfa_debug.so
+LIB_PATH = os.environ.get("FA_LIBRARY") or os.path.join(_HERE, "libfa.so")
 
 FA_OK = 0
 FA_ERR_INVALID = 1
@@ -26,6 +27,7 @@ FA_ERR_WORKSPACE = 3
 FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
 FA_ERR_DEVICE_ARG = 6
+FA_ERR_DEBUG_CHECK = 7
 FA_BF16 = 0
 FA_F32 = 1
 
@@ -50,6 +52,8 @@ SIGNATURES = {
     "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "fa_fwd_selftest_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_decode_selftest_timeout": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "fa_build_flags": (_I, []),
+    "fa_debug_selftest_bounds": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_status_str": (ctypes.c_char_p, [_I]),
     "fa_last_error_message": (ctypes.c_char_p, []),
     "fa_version": (_I, []),

@@ -49,8 +49,10 @@ typedef enum {
     FA_ERR_WORKSPACE = 3,    /* decode workspace null or smaller than required */
     FA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed; see fa_last_error_message */
     FA_ERR_TIMEOUT = 5,      /* a kernel pipeline wait exceeded its time limit (fa_get_error) */
-    FA_ERR_DEVICE_ARG = 6    /* the device found seqlens[b] outside [0, Nmax] and clamped it,
+    FA_ERR_DEVICE_ARG = 6,   /* the device found seqlens[b] outside [0, Nmax] and clamped it,
                                 or a block-table entry outside the page pool */
+    FA_ERR_DEBUG_CHECK = 7   /* debug builds only: a global-memory index computed by a kernel
+                                failed its bounds check; the access was skipped */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
@@ -271,7 +273,8 @@ FA_API int fa_decode_noalloc(const void *q, const void *kcache, const void *vcac
 
 /*
  * Synchronises `stream`, then reads and clears the device error word.  Returns FA_OK,
- * FA_ERR_TIMEOUT, FA_ERR_DEVICE_ARG, or FA_ERR_CUDA if the synchronisation itself failed.
+ * FA_ERR_TIMEOUT, FA_ERR_DEVICE_ARG, FA_ERR_DEBUG_CHECK (debug builds), or FA_ERR_CUDA if
+ * the synchronisation itself failed.
  */
 FA_API int fa_get_error(void *stream);
 
@@ -307,6 +310,26 @@ FA_API int fa_decode_selftest_timeout(const void *q, const void *kcache, const v
                                       const float *k_scale, const float *v_scale, const int *seqlens,
                                       void *o, float *lse, int B, int Hq, int Hkv, int Nmax, int d,
                                       float scale, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Build flags of this library: bit 0 set in the debug build (libfa_debug.so, compiled with
+ * FA_DEBUG_CHECKS), whose kernels check every global-memory index they compute by hand
+ * (outputs, decode partials, scales, q rows, block-table entries) against the size of its
+ * buffer, skip the access on a failure and report FA_ERR_DEBUG_CHECK through fa_get_error.
+ * The results are the release build's; only speed differs.
+ */
+FA_API int fa_build_flags(void);
+
+/*
+ * Self-test of the debug build's bounds checks: runs the prefill of fa_fwd on the given
+ * (valid) arguments with every LSE index moved out of its buffer, so each LSE store must
+ * fail its check and be skipped (lse is left as it was; O is computed normally);
+ * fa_get_error afterwards returns FA_ERR_DEBUG_CHECK.  In a release build (no checks
+ * compiled in) it returns FA_ERR_UNSUPPORTED and launches nothing.
+ */
+FA_API int fa_debug_selftest_bounds(const void *q, const void *k, const void *v, void *o, float *lse,
+                                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                                    int causal, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 FA_API const char *fa_status_str(int status);
