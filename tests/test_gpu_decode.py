@@ -31,6 +31,8 @@ CASES = [  # (B, Hq, Hkv, Nmax, d, lengths)
     (2, 6, 2, 700, 128, [700, 3]),                  # R=3
     (2, 12, 2, 600, 64, [600, 512]),                # R=6
     (1, 32, 8, 8192, 128, [8192]),                  # one full-length sequence
+    (2, 8, 1, 65536, 128, [65536, 40000]),          # 256 splits per sequence into the merge
+    (3, 1, 1, 900, 64, [900, 1, 450]),              # a single head
 ]
 
 

@@ -53,6 +53,10 @@ SMALL = [  # (B, Hq, Hkv, Nq, Nk, d, causal)
     (1, 2, 1, 255, 255, 128, True),
     (2, 2, 2, 513, 513, 128, True),
     (1, 16, 2, 384, 384, 128, True),    # R=8
+    (64, 16, 16, 64, 64, 128, True),    # 1024 short work slots over the persistent CTAs
+    (64, 16, 16, 64, 64, 64, False),
+    (1, 4, 2, 1, 5000, 128, False),     # one query row against a long key range
+    (2, 8, 8, 3, 2000, 64, True),       # three new rows at the end of a long context
 ]
 
 
