@@ -84,9 +84,14 @@ def load_traffic():
 # ------------------------------------------------------------------ clocks sampler
 
 class ClockSampler:
-    """Samples SM clock, power and clock-event reasons through NVML in a thread."""
+    """Samples SM clock, power and clock-event reasons through NVML in a thread.
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    The clock and the reasons are read every ``period_s`` (a few samples fall inside even a
+    timed region of well under a second); the power reading, the slowest of the three
+    calls, only on every fourth sample (the last reading is repeated in between).
+    """
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.period = period_s
         self.samples = []
         self.ok = False
@@ -124,6 +129,7 @@ class ClockSampler:
 
     def _run(self):
         nv = self.nv
+        pw, n = 0.0, 0
         while not self._stop.is_set():
             try:
                 mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
@@ -131,7 +137,9 @@ class ClockSampler:
                     mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
                 except Exception:
                     mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
-                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                if n % 4 == 0:
+                    pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                n += 1
                 self.samples.append((time.time(), mhz, pw, self._reasons(mask)))
             except Exception:
                 pass
