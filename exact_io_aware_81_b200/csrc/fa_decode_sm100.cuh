@@ -53,7 +53,7 @@
 //     output dims; one byte permute per register puts them in the order (0, 2, 1, 3) so
 //     that its two halves convert directly.  P is converted to fp16 and v_scale is applied
 //     with the final 1 / l.
-// (Measured on B200: the hardware conversion for K and V is 6% faster on the FP8 decode
+// (Measured on B200: the hardware conversion for K and V is 7% faster on the FP8 decode
 // workload than moving the E4M3 bit fields into fp16 with integer operations, whose
 // arithmetic kept the ALU pipe the busiest unit of the kernel.)
 #pragma once
